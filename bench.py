@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Throughput of the B200 Mixtral sparse-MoE layer (route -> dispatch -> experts -> combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skew|quarter|tiny]
+                    [--impl ours|reference]
+
+One step = one forward of the whole layer over one batch of T synthetic tokens
+(Mixtral 8x7B shapes: d=4096, d_ff=14336, E=8, k=2), inputs resident in HBM.
+Timing: CUDA events on the launching stream around each step, W warm-up steps,
+512 MiB written between timed steps to flush the 126 MB L2; the per-step device
+time excludes the flush.  N > 1 (torchrun): every rank runs an independent
+replica on its own GPU (no collective on the data path); the reported time is
+the max over ranks and `value` counts the tokens of all ranks.
+
+`--impl reference` times the CPU oracle (oracle/, plain C, fp64) on a bounded
+sample of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; % of BF16 TC peak (prefill), % of HBM GB/s (decode)"
+WORKLOAD_NAMES = {
+    "prefill": "mixtral-8x7b-moe-prefill T=4096",
+    "decode": "mixtral-8x7b-moe-decode T=16",
+    "skew": "mixtral-8x7b-moe-prefill-skewed T=16384",
+    "quarter": "quarter-width-moe T=1024 d=1024 d_ff=3584",
+    "tiny": "tiny-moe T=64 d=128 d_ff=256",
+}
+FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+KERNEL_SOURCES = ["sparse_mixture_experts_05_b200/csrc/expert_gemm.cu",
+                  "sparse_mixture_experts_05_b200/csrc/sm100.cuh"]
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill", choices=list(WORKLOAD_NAMES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the decode-workload line added to the prefill run")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload):
+    """DRAM bytes per launch of the expert kernel from the committed ncu summary, when it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_sha") != source_hash():
+        return None
+    return t.get("per_step_bytes", {}).get(workload)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if __import__("torch").cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    return world, rank, local, pg
+
+
+def reduce_max(pg, value: float, device) -> float:
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device):
+    if pg is None:
+        return
+    import torch
+    t = torch.zeros(1, device=device)
+    pg.all_reduce(t)
+
+
+# ---------------------------------------------------------------- our arm
+def algorithmic(shape, counts):
+    T, d, d_ff, E, k = shape
+    R = T * k
+    flops_experts = 6 * R * d * d_ff
+    flops_router = 2 * T * d * E
+    touched = sum(1 for c in counts if c > 0)
+    weight_bytes = touched * 3 * d * d_ff * 2
+    return {
+        "flops_gemm1": 4 * R * d * d_ff,
+        "flops_gemm2": 2 * R * d * d_ff,
+        "flops_total": flops_experts + flops_router,
+        "bytes_expert_weights": weight_bytes,
+        # bytes each memory-bound kernel must move at least once
+        "bytes_router": T * d * 2 + d * E * 2 + T * k * 8,
+        "bytes_dispatch": T * k * 4 * 3 + T * d * 2 + R * d * 2,
+        "bytes_combine": R * d * 4 + T * d * 2 + T * k * 8,
+        # decode: the experts' weights plus their activations
+        "bytes_experts_decode": weight_bytes + R * d * 2 + R * d_ff * 2 * 2 + R * d * 4,
+    }
+
+
+def time_workload(name, steps, warmup, device, rank):
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    from sparse_mixture_experts_05_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS[name]
+    inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
+    shape = inp["shape"]
+    x, Wg, bias, W1, W3, W2 = (inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
+    ws = moe.workspace(moe.moe_forward_workspace_bytes(shape), device)
+    y = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    n_ev = len(moe.binding.PROFILE_EVENTS)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
+    for row in events:
+        for ev in row:
+            ev.record()
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for ev in warm:
+        ev.record()
+    for _ in range(warmup):
+        moe.moe_forward_profiled(shape, x, Wg, bias, W1, W3, W2, warm, y=y, ws=ws)
+    torch.cuda.synchronize()
+    status = moe.moe_read_device_status(ws)
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {moe.status_string(status)}")
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=device)
+    moe.moe_forward(shape, x, Wg, bias, W1, W3, W2, y=y, idx_out=idx, ws=ws)
+    counts = torch.bincount(idx.flatten().long(), minlength=w.E).tolist()
+
+    return dict(inp=inp, shape=shape, ws=ws, y=y, flush=flush, events=events, counts=counts,
+                run=lambda i: moe.moe_forward_profiled(shape, x, Wg, bias, W1, W3, W2, events[i],
+                                                       y=y, ws=ws))
+
+
+def timed_loop(ctx, steps, pg, device, clock):
+    import torch
+    barrier(pg, device)
+    torch.cuda.synchronize()
+    clock.start()
+    outer0 = torch.cuda.Event(enable_timing=True)
+    outer1 = torch.cuda.Event(enable_timing=True)
+    outer0.record()
+    for i in range(steps):
+        ctx["flush"].fill_(i & 0xFF)
+        ctx["run"](i)
+    outer1.record()
+    torch.cuda.synchronize()
+    barrier(pg, device)
+    clocks = clock.stop()
+    ev = ctx["events"]
+    step_ms = [ev[i][0].elapsed_time(ev[i][6]) for i in range(steps)]
+    parts = {}
+    import sparse_mixture_experts_05_b200 as moe
+    names = moe.binding.PROFILE_EVENTS
+    for j in range(1, len(names)):
+        parts[names[j]] = sum(ev[i][j - 1].elapsed_time(ev[i][j]) for i in range(steps)) / steps
+    return step_ms, parts, outer0.elapsed_time(outer1), clocks
+
+
+def e2e_loop(ctx, steps, warmup, device):
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    inp = ctx["inp"]
+    shape = ctx["shape"]
+    T, d = shape[0], shape[1]
+    ws = moe.workspace(moe.moe_forward_hostio_workspace_bytes(shape), device)
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    args = (shape, x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, ws)
+    for _ in range(warmup):
+        moe.moe_forward_hostio(*args)
+    torch.cuda.synchronize()
+    ms = []
+    for i in range(steps):
+        ctx["flush"].fill_(i & 0xFF)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        moe.moe_forward_hostio(*args)
+        b.record()
+        b.synchronize()
+        _ = float(y_host[0, 0])  # the host reads the step's result
+        ms.append(a.elapsed_time(b))
+    if moe.moe_read_device_status(ws) != moe.MOE_OK:
+        raise RuntimeError("device status error in the end-to-end loop")
+    return statistics.mean(ms), T * d * 2, T * d * 2
+
+
+def oracle_sample(inp, seconds, device_inputs=True):
+    """Times the oracle's per-token forward on a sample of tokens; returns dict."""
+    import numpy as np
+
+    import oracle
+    T, d, d_ff, E, k = inp["shape"]
+    host = {key: (inp[key].cpu() if inp[key] is not None else None)
+            for key in ("x", "Wg", "bias", "W1", "W3", "W2")}
+    oracle.build()
+    rng = np.random.default_rng(0)
+    t0 = time.perf_counter()
+    oracle.forward_tokens(np.array([0], np.int32), host["x"], host["Wg"], host["W1"], host["W3"],
+                          host["W2"], k, bias=host["bias"])
+    one = max(time.perf_counter() - t0, 1e-4)
+    cores = os.cpu_count() or 1
+    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    n = int(max(1, min(T, 4096, seconds / one * min(threads, 64) * 0.8)))
+    toks = np.sort(rng.choice(T, n, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.forward_tokens(toks, host["x"], host["Wg"], host["W1"], host["W3"], host["W2"], k,
+                          bias=host["bias"])
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of the workload's {T} tokens, per-token oracle loop (route, 2 SwiGLU "
+                      f"experts, combine) in fp64, {dt:.1f} s wall"}, host
+
+
+def run_ours(a):
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    world, rank, local, pg = dist_setup(a.gpus)
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    peaks, peak_kind = load_peaks()
+    moe.binding.lib()
+
+    ctx = time_workload(a.workload, a.steps, a.warmup, device, rank)
+    clock = ClockSampler(local)
+    step_ms, parts, bracket_ms, clocks = timed_loop(ctx, a.steps, pg, device, clock)
+    mean_ms = statistics.mean(step_ms)
+    max_ms = reduce_max(pg, mean_ms, device)
+    shape = ctx["shape"]
+    T = shape[0]
+    alg = algorithmic(shape, ctx["counts"])
+    value = T * world / (max_ms / 1000.0)
+
+    e2e_ms, h2d, d2h = e2e_loop(ctx, a.steps, a.warmup, device)
+    e2e_ms = reduce_max(pg, e2e_ms, device)
+
+    gemm_ms = parts["gemm1_swiglu"] + parts["gemm2_down"]
+    flops_e = alg["flops_gemm1"] + alg["flops_gemm2"]
+    if a.workload in ("decode",):
+        achieved = alg["bytes_experts_decode"] / (gemm_ms / 1000) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                "frac_of_spec_8000": round(achieved / SPEC_HBM_GBS, 4)}
+    else:
+        achieved = flops_e / (gemm_ms / 1000) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_kind": f"{peak_kind} burst bf16 GEMM",
+                "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
+                "frac_of_spec_2250": round(achieved / SPEC_BF16_TFLOPS, 4)}
+    roof["kernel"] = ("expert_gemm_kernel (two launches per step: GEMM1 x.W1|x.W3 -> SiLU(a)*b, "
+                      "GEMM2 h.W2); achieved = algorithmic units of both launches / their summed "
+                      "CUDA-event time")
+    traffic = committed_traffic(a.workload)
+    roof["traffic"] = traffic
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(max_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) tokens and N(0,1/fan_in) bf16 weights (no dataset, "
+                "no trained weights)",
+        "config": {"workload": WORKLOAD_NAMES[a.workload], "model": "Mixtral 8x7B MoE layer",
+                   "T": T, "d": shape[1], "d_ff": shape[2], "E": shape[3], "k": shape[4],
+                   "global_batch": T * world, "seq_len": T, "parallelism": f"replicas x{world}",
+                   "l2": "flushed: 512 MiB written between timed steps (flush not timed)",
+                   "expert_rows": ctx["counts"]},
+        "roofline": roof,
+        "e2e": {"value": round(T * world / (e2e_ms / 1000.0), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "moe_forward_hostio (pinned host x -> device -> layer -> host y)"},
+        "gpu_launches": 6 * a.steps,
+        "clocks": clocks,
+        "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
+        "tflops_layer": round(alg["flops_total"] / (max_ms / 1000) / 1e12, 1),
+        "bracket_ms_incl_flush": round(bracket_ms, 3),
+    }
+    del ctx
+    torch.cuda.empty_cache()
+
+    if a.workload == "prefill" and not a.no_secondary:
+        dctx = time_workload("decode", a.steps, a.warmup, device, rank)
+        d_ms, d_parts, _, d_clocks = timed_loop(dctx, a.steps, pg, device, ClockSampler(local))
+        d_mean = reduce_max(pg, statistics.mean(d_ms), device)
+        d_alg = algorithmic(dctx["shape"], dctx["counts"])
+        d_gemm = d_parts["gemm1_swiglu"] + d_parts["gemm2_down"]
+        d_gbs = d_alg["bytes_experts_decode"] / (d_gemm / 1000) / 1e9
+        line["decode"] = {
+            "workload": WORKLOAD_NAMES["decode"], "tokens_per_s": round(16 * world / (d_mean / 1e3), 1),
+            "ms_per_step": round(d_mean, 4),
+            "experts_gbs": round(d_gbs, 1), "frac_of_measured_hbm": round(d_gbs / peaks["hbm_gbs"], 4),
+            "frac_of_spec_8000": round(d_gbs / SPEC_HBM_GBS, 4),
+            "layer_gbs": round((d_alg["bytes_experts_decode"] + d_alg["bytes_router"]) /
+                               (d_mean / 1000) / 1e9, 1),
+            "kernel_ms": {k_: round(v, 4) for k_, v in d_parts.items()},
+            "expert_rows": dctx["counts"], "clocks": d_clocks}
+        if world == 1 and rank == 0 and not a.no_cpu_baseline:
+            pass
+        del dctx
+        torch.cuda.empty_cache()
+
+    if world == 1 and rank == 0 and not a.no_cpu_baseline:
+        from sparse_mixture_experts_05_b200.inputs import WORKLOADS, make_inputs
+        w = WORKLOADS[a.workload]
+        inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
+        cb, _ = oracle_sample(inp, a.cpu_seconds)
+        line["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------- reference arm (CPU oracle)
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from sparse_mixture_experts_05_b200.inputs import WORKLOADS, make_inputs
+    import numpy as np
+
+    import oracle
+    w = WORKLOADS[a.workload]
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
+    host = {key: (inp[key].cpu() if inp[key] is not None else None)
+            for key in ("x", "Wg", "bias", "W1", "W3", "W2")}
+    oracle.build()
+    T, k = w.T, w.k
+    t0 = time.perf_counter()
+    oracle.forward_tokens(np.array([0], np.int32), host["x"], host["Wg"], host["W1"], host["W3"],
+                          host["W2"], k, bias=host["bias"])
+    one = max(time.perf_counter() - t0, 1e-4)
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    budget = 150.0 / (a.steps + a.warmup)  # whole run within a few minutes
+    n = int(max(1, min(T, budget / one * min(threads, 64) * 0.7)))
+    rng = np.random.default_rng(1)
+    times = []
+    for i in range(a.warmup + a.steps):
+        toks = np.sort(rng.choice(T, n, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.forward_tokens(toks, host["x"], host["Wg"], host["W1"], host["W3"], host["W2"], k,
+                              bias=host["bias"])
+        if i >= a.warmup:
+            times.append(time.perf_counter() - t0)
+    step_s = statistics.mean(times)
+    value = n / step_s
+    sample = (f"{n} random tokens of the workload's {T} per step, per-token oracle loop in fp64 "
+              f"(route, k SwiGLU experts, combine)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(step_s * 1000, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe and seeds)",
+        "config": {"workload": WORKLOAD_NAMES[a.workload], "model": "Mixtral 8x7B MoE layer",
+                   "T": T, "d": w.d, "d_ff": w.d_ff, "E": w.E, "k": w.k,
+                   "global_batch": T, "seq_len": T, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    a = parse(argv)
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,200 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Mixtral sparse-MoE feed-forward layer.
+ *
+ * The layer (Mixtral textbook page, llm-arch-research, section "Прямой проход в
+ * формулах", the MoE equation; the same formula in section "Научный вклад"):
+ *
+ *     g = u W_r,   S = TopK(g, k),   w_i = exp(g_i) / sum_{j in S} exp(g_j),
+ *     MoE(u) = sum_{i in S} w_i * (SiLU(u W1_i) (.) (u W3_i)) W2_i
+ *
+ * computed, as in that page's section "Алгоритм" (algorithm), as a loop over
+ * experts rather than tokens: route every token, list each expert's tokens
+ * (dispatch), run each expert once over its rows, and add each token's k
+ * gate-weighted expert outputs (combine).  No capacity limit, no dropped
+ * tokens: every token gets exactly k terms and the experts process T*k rows.
+ *
+ * Conventions for every entry point
+ *  - Layouts are row-major and dense.  bf16 tensors are passed as raw 16-bit
+ *    storage (void*).  Shapes:
+ *        x        [T, d]        bf16   tokens (already normalised: the layer input u)
+ *        Wg       [d, E]        bf16   router W_r (E fastest)
+ *        bias     [E]           float  optional router bias (nullable)
+ *        W1, W3   [E, d, d_ff]  bf16   gate / up projections (u W1_e, u W3_e)
+ *        W2       [E, d_ff, d]  bf16   down projection
+ *        y        [T, d]        bf16   layer output
+ *  - Every pointer except `stream` is DEVICE memory owned by the caller, except
+ *    in moe_forward_hostio where x and y are HOST memory.  The library never
+ *    allocates or frees memory and never synchronises, except
+ *    moe_read_device_status (documented there).  All work is enqueued
+ *    asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *    on the current device.
+ *  - Every pointer must be 16-byte aligned.
+ *  - Arguments are checked on the host before anything is launched; a failed
+ *    check returns a non-zero status and launches nothing (the counterpart of
+ *    the ValueError the page's MoE constructor raises for a top_k_experts
+ *    outside 1..num_experts, section "Mixtral" / "Конфигурация").
+ *  - Supported shapes: T >= 0 (T == 0 is a no-op), 1 <= k <= E <= 32, k <= 8,
+ *    d and d_ff multiples of 128, T*k*max(d, d_ff) < 2^31, and
+ *    16 * d * ceil(E/8) <= 163840 (router tile in shared memory).
+ *
+ * Precision: bf16 inputs, fp32 accumulation on tensor cores; router logits,
+ * gates and expert outputs o in fp32; the SwiGLU product h stored in bf16 (the
+ * down projection's tensor-core input); y rounded once to bf16 (nearest-even).
+ * Top-k ties go to the lower expert index; slot 0 holds the largest logit.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, k outside 1..E, negative size */
+    MOE_ERR_UNSUPPORTED = 2,    /* legal shape this build does not handle (see limits above) */
+    MOE_ERR_WORKSPACE = 3,      /* workspace smaller than the matching *_workspace_bytes */
+    MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait expired (see moe_read_device_status) */
+} moe_status;
+
+typedef struct {
+    int32_t T;     /* tokens (batch * seq_len, the page's N = batch * seq_len) */
+    int32_t d;     /* model width (emb_size) */
+    int32_t d_ff;  /* expert hidden width (intermediate_size) */
+    int32_t E;     /* experts (num_experts) */
+    int32_t k;     /* experts per token (top_k_experts) */
+} moe_shape;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(int status);
+
+/* Checks a shape against the limits above without touching the GPU. */
+int moe_check_shape(moe_shape s);
+
+/* Bytes of workspace moe_expert_swiglu needs for shape s (status word and
+ * scheduling state). */
+size_t moe_expert_workspace_bytes(moe_shape s);
+
+/* Bytes of workspace moe_forward / moe_forward_hostio need for shape s (every
+ * intermediate of the layer plus the moe_expert_swiglu workspace). */
+size_t moe_forward_workspace_bytes(moe_shape s);
+
+/*
+ * moe_route -- router, top-k and softmax over the selected k.
+ * Page: section "Прямой проход в формулах" (g = u W_r, S = TopK(g, k), w_i) and
+ * section "MoE изнутри" (softmax over the k selected logits, in float32).
+ *   x [T,d] bf16, Wg [d,E] bf16, bias [E] float or NULL  (in)
+ *   idx [T,k] int32   expert ids, slot 0 = largest logit, ties -> lower id (out)
+ *   gate [T,k] float  w_i of the selected experts, summing to 1 (out)
+ *   logits [T,E] float  g (+ bias) in float32, or NULL (out)
+ */
+int moe_route(moe_shape s, const void* x, const void* Wg, const float* bias, int32_t* idx,
+              float* gate, float* logits, void* stream);
+
+/*
+ * moe_dispatch -- per-expert token lists (dispatch of section "Алгоритм":
+ * tok, slot = where(topk_idx == e), in ascending token order).
+ *   idx [T,k] int32 (in), x [T,d] bf16 (in)
+ *   offsets [E+1] int32: rows of expert e are offsets[e] .. offsets[e+1]-1 (out)
+ *   perm_tok [T*k] int32: token of each sorted row (out)
+ *   inv [T,k] int32: sorted row of each (token, slot); -1 if idx was outside 0..E-1 (out)
+ *   x_sorted [T*k,d] bf16: x_sorted[r] = x[perm_tok[r]] (out)
+ * Entries of idx outside 0..E-1 get no row; then offsets[E] < T*k.
+ */
+int moe_dispatch(moe_shape s, const int32_t* idx, const void* x, int32_t* offsets,
+                 int32_t* perm_tok, int32_t* inv, void* x_sorted, void* stream);
+
+/*
+ * moe_expert_swiglu -- Expert_e(X[tok]) for every expert e over its rows
+ * (section "Алгоритм"; expert = SwiGLU of section "Прямой проход в формулах").
+ *   x_sorted [T*k,d] bf16, offsets [E+1] int32 (from moe_dispatch) (in)
+ *   W1, W3 [E,d,d_ff] bf16, W2 [E,d_ff,d] bf16 (in)
+ *   h [T*k,d_ff] bf16: SiLU(x W1_e) (.) (x W3_e), rounded to bf16 (out)
+ *   o [T*k,d] float:   h W2_e (out)
+ *   ws: >= moe_expert_workspace_bytes(s) bytes of device memory (scratch)
+ * Rows at or beyond offsets[E] are left untouched; an expert without rows
+ * costs nothing.  A device wait that expires leaves o/h incomplete and is
+ * reported by moe_read_device_status(ws).
+ */
+int moe_expert_swiglu(moe_shape s, const void* x_sorted, const int32_t* offsets, const void* W1,
+                      const void* W3, const void* W2, void* h, float* o, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_swiglu_stall_test -- test hook for the error path of the bounded
+ * device waits (no counterpart on the pages).  Runs moe_expert_swiglu with its
+ * TMA producer stopping after `stall_after` (>= 0) pipeline stages, as if it had
+ * died, and every device wait bounded by `timeout_ns` (1e3 .. 2e9).  The waiting
+ * roles give up after timeout_ns, drain their copies and MMAs, free tensor
+ * memory and return; moe_read_device_status(ws) then reports
+ * MOE_ERR_DEVICE_TIMEOUT and the CUDA context stays usable.  h and o are left
+ * incomplete.
+ */
+int moe_expert_swiglu_stall_test(moe_shape s, const void* x_sorted, const int32_t* offsets,
+                                 const void* W1, const void* W3, const void* W2, void* h, float* o,
+                                 void* ws, size_t ws_bytes, int stall_after,
+                                 uint64_t timeout_ns, void* stream);
+
+/*
+ * moe_combine -- y[t] = sum over slots s (in slot order) of gate[t,s] * o[inv[t,s]]
+ * (combine of section "Алгоритм": Y.index_add_(0, tok, W[tok,slot] * Expert_e(X[tok]))).
+ * Products and sums in float32 without fused multiply-add; y rounded to bf16.
+ *   o [T*k,d] float, inv [T,k] int32, gate [T,k] float (in);  y [T,d] bf16 (out)
+ * Slots with inv < 0 are skipped.
+ */
+int moe_combine(moe_shape s, const float* o, const int32_t* inv, const float* gate, void* y,
+                void* stream);
+
+/*
+ * moe_forward -- the whole layer: route, dispatch, experts, combine.
+ *   x, Wg, bias (nullable), W1, W3, W2 as above (in);  y [T,d] bf16 (out)
+ *   idx_out [T,k] int32, gate_out [T,k] float: copies of the routing, or NULL
+ *   ws: >= moe_forward_workspace_bytes(s) bytes of device memory
+ */
+int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, const void* W1,
+                const void* W3, const void* W2, void* y, int32_t* idx_out, float* gate_out,
+                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_forward_profiled -- moe_forward (no idx/gate copies) that also records
+ * seven caller-created CUDA events (cudaEvent_t handles) on `stream` between its
+ * launches: events[0] before the router, [1] after the router, [2] after the
+ * dispatch index kernel, [3] after the dispatch scatter, [4] after GEMM1
+ * (x W1 | x W3 -> h), [5] after GEMM2 (h W2 -> o), [6] after the combine.
+ * n_events must be 7.  Measurement hook with no counterpart on the pages.
+ */
+int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float* bias,
+                         const void* W1, const void* W3, const void* W2, void* y, void* ws,
+                         size_t ws_bytes, void* const* events, int n_events, void* stream);
+
+/*
+ * moe_forward_hostio -- moe_forward with x and y in HOST memory (pinned memory
+ * gives asynchronous copies): enqueues the host->device copy of x into the
+ * workspace, the layer, and the device->host copy of y, all on `stream`.  The
+ * caller synchronises the stream before reading y.  Weights stay on the device.
+ *   ws: >= moe_forward_workspace_bytes(s) + T*d*2 (x staging) + T*d*2 (y staging)
+ *       bytes; moe_forward_hostio_workspace_bytes gives the exact figure.
+ */
+size_t moe_forward_hostio_workspace_bytes(moe_shape s);
+int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const float* bias,
+                       const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/*
+ * moe_read_device_status -- SYNCHRONISES `stream`, then reads the status word
+ * that moe_expert_swiglu / moe_forward keep at the start of their workspace:
+ * MOE_OK, or MOE_ERR_DEVICE_TIMEOUT when a bounded device wait gave up
+ * (the kernel then stopped issuing work, drained its copies, freed its tensor
+ * memory and returned).  The word is reset by the next call that uses `ws`.
+ */
+int moe_read_device_status(const void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,288 @@
+// api.cu -- the C ABI declared in include/moe.h: argument checks, workspace
+// carving and the launch sequence of the MoE layer.
+//
+// The launch sequence follows the loop of the Mixtral textbook page, section
+// "Алгоритм": route (topk of X W_r, softmax over the k), dispatch (per-expert
+// token lists), experts (one grouped pass per GEMM over all expert groups),
+// combine (k gate-weighted terms per token).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "expert_gemm.cuh"
+#include "router.cuh"
+
+namespace moe {
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+int check_shape(const moe_shape& s) {
+    if (s.T < 0 || s.d <= 0 || s.d_ff <= 0 || s.E <= 0 || s.k <= 0) return MOE_ERR_INVALID_ARG;
+    if (s.k > s.E) return MOE_ERR_INVALID_ARG;  // top_k_experts must lie in 1 .. num_experts
+    if (s.E > 32 || s.k > 8) return MOE_ERR_UNSUPPORTED;
+    if (s.d % 128 != 0 || s.d_ff % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    const int64_t R = (int64_t)s.T * s.k;
+    if (R * (int64_t)std::max(s.d, s.d_ff) >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)s.E * std::max(s.d, s.d_ff) >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)16 * s.d * ((s.E + 7) / 8) > 163840) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+
+// Workspace of moe_forward, in order; every segment starts on a 256-byte boundary.
+struct FwdLayout {
+    size_t hdr, idx, gate, offsets, perm, inv, x_sorted, h, o, total;
+};
+
+FwdLayout fwd_layout(const moe_shape& s) {
+    const size_t T = (size_t)s.T, R = (size_t)s.T * s.k;
+    FwdLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, kAlign);
+        return at;
+    };
+    L.hdr = take(kWsHeaderBytes);
+    L.idx = take(T * s.k * 4);
+    L.gate = take(T * s.k * 4);
+    L.offsets = take((size_t)(s.E + 1) * 4);
+    L.perm = take(R * 4);
+    L.inv = take(R * 4);
+    L.x_sorted = take(R * s.d * 2);
+    L.h = take(R * s.d_ff * 2);
+    L.o = take(R * s.d * 4);
+    L.total = off;
+    return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+constexpr int kProfileEvents = 7;
+
+// Records events[i] (when given) between the launches: 0 before the router, 1
+// after it, 2 after the dispatch index kernel, 3 after the scatter, 4 after
+// GEMM1, 5 after GEMM2, 6 after the combine.
+int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias,
+                 const void* W1, const void* W3, const void* W2, void* y, int32_t* idx_out,
+                 float* gate_out, void* ws, cudaStream_t st, void* const* events) {
+    auto mark = [&](int i) {
+        return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
+    };
+    const FwdLayout L = fwd_layout(s);
+    int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+    float* gate = gate_out ? gate_out : at<float>(ws, L.gate);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* perm = at<int32_t>(ws, L.perm);
+    int32_t* inv = at<int32_t>(ws, L.inv);
+    void* xs = at<void>(ws, L.x_sorted);
+    void* h = at<void>(ws, L.h);
+    float* o = at<float>(ws, L.o);
+    int* status = at<int>(ws, L.hdr);
+    if (!mark(0)) return MOE_ERR_CUDA;
+    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st);
+    if (rc) return rc;
+    if (!mark(1)) return MOE_ERR_CUDA;
+    rc = launch_dispatch_index(s, idx, offsets, perm, inv, status, st);
+    if (rc) return rc;
+    if (!mark(2)) return MOE_ERR_CUDA;
+    rc = launch_dispatch_scatter(s, x, inv, xs, st);
+    if (rc) return rc;
+    if (!mark(3)) return MOE_ERR_CUDA;
+    rc = expert_gemms(s, xs, offsets, W1, W3, W2, h, o, status, kDefaultWaitTimeoutNs, -1, st,
+                      events ? events[4] : nullptr);
+    if (rc) return rc;
+    if (!mark(5)) return MOE_ERR_CUDA;
+    rc = launch_combine(s, o, inv, gate, y, st);
+    if (rc) return rc;
+    return mark(6) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument (null/misaligned pointer, k outside 1..E, negative size)";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape outside the supported limits";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a bounded device-side wait expired";
+        default: return "unknown moe status";
+    }
+}
+
+int moe_check_shape(moe_shape s) { return check_shape(s); }
+
+size_t moe_expert_workspace_bytes(moe_shape s) {
+    if (check_shape(s)) return 0;
+    return kWsHeaderBytes;
+}
+
+size_t moe_forward_workspace_bytes(moe_shape s) {
+    if (check_shape(s)) return 0;
+    return fwd_layout(s).total;
+}
+
+size_t moe_forward_hostio_workspace_bytes(moe_shape s) {
+    if (check_shape(s)) return 0;
+    const size_t io = align_up((size_t)s.T * s.d * 2, 256);
+    return fwd_layout(s).total + 2 * io;
+}
+
+int moe_route(moe_shape s, const void* x, const void* Wg, const float* bias, int32_t* idx,
+              float* gate, float* logits, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(idx) || !ok_ptr(gate) ||
+        !ok_opt(logits))
+        return MOE_ERR_INVALID_ARG;
+    return launch_router(s, x, Wg, bias, idx, gate, logits, static_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch(moe_shape s, const int32_t* idx, const void* x, int32_t* offsets,
+                 int32_t* perm_tok, int32_t* inv, void* x_sorted, void* stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
+    if (s.T > 0 && (!ok_ptr(idx) || !ok_ptr(x) || !ok_ptr(perm_tok) || !ok_ptr(inv) ||
+                    !ok_ptr(x_sorted)))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_dispatch_index(s, idx, offsets, perm_tok, inv, nullptr, st);
+    if (rc) return rc;
+    return launch_dispatch_scatter(s, x, inv, x_sorted, st);
+}
+
+int moe_expert_swiglu(moe_shape s, const void* x_sorted, const int32_t* offsets, const void* W1,
+                      const void* W3, const void* W2, void* h, float* o, void* ws,
+                      size_t ws_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x_sorted) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(h) || !ok_ptr(o) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_expert_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return MOE_ERR_CUDA;
+    return expert_gemms(s, x_sorted, offsets, W1, W3, W2, h, o, static_cast<int*>(ws),
+                        kDefaultWaitTimeoutNs, -1, st, nullptr);
+}
+
+int moe_expert_swiglu_stall_test(moe_shape s, const void* x_sorted, const int32_t* offsets,
+                                 const void* W1, const void* W3, const void* W2, void* h, float* o,
+                                 void* ws, size_t ws_bytes, int stall_after,
+                                 uint64_t timeout_ns, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x_sorted) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(h) || !ok_ptr(o) || !ok_ptr(ws) || stall_after < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (timeout_ns < 1000 || timeout_ns > kDefaultWaitTimeoutNs) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_expert_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return MOE_ERR_CUDA;
+    return expert_gemms(s, x_sorted, offsets, W1, W3, W2, h, o, static_cast<int*>(ws), timeout_ns,
+                        stall_after, st, nullptr);
+}
+
+int moe_combine(moe_shape s, const float* o, const int32_t* inv, const float* gate, void* y,
+                void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(o) || !ok_ptr(inv) || !ok_ptr(gate) || !ok_ptr(y)) return MOE_ERR_INVALID_ARG;
+    return launch_combine(s, o, inv, gate, y, static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, const void* W1,
+                const void* W3, const void* W2, void* y, int32_t* idx_out, float* gate_out,
+                void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(y) || !ok_opt(idx_out) || !ok_opt(gate_out) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    return forward_impl(s, x, Wg, bias, W1, W3, W2, y, idx_out, gate_out, ws,
+                        static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float* bias,
+                         const void* W1, const void* W3, const void* W2, void* y, void* ws,
+                         size_t ws_bytes, void* const* events, int n_events, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(y) || !ok_ptr(ws) || !events || n_events != kProfileEvents)
+        return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < kProfileEvents; ++i)
+        if (!events[i]) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    return forward_impl(s, x, Wg, bias, W1, W3, W2, y, nullptr, nullptr, ws,
+                        static_cast<cudaStream_t>(stream), events);
+}
+
+int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const float* bias,
+                       const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
+                       size_t ws_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!x_host || !y_host || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) ||
+        !ok_ptr(W2) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_hostio_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t fwd = moe_forward_workspace_bytes(s);
+    const size_t io_bytes = (size_t)s.T * s.d * 2;
+    void* x_dev = static_cast<char*>(ws) + fwd;
+    void* y_dev = static_cast<char*>(ws) + fwd + align_up(io_bytes, 256);
+    if (cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    rc = forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st, nullptr);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(y_host, y_dev, io_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int moe_read_device_status(const void* ws, void* stream) {
+    if (!ok_ptr(ws)) return MOE_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (word == 0) return MOE_OK;
+    if (word & kDeviceTimeoutBase) return MOE_ERR_DEVICE_TIMEOUT;
+    return MOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,437 @@
+// expert_gemm.cu -- grouped expert GEMMs on the 5th-generation tensor cores.
+//
+// The experts of the MoE layer (Mixtral textbook page, section "Прямой проход в
+// формулах": Expert_i(u) = (SiLU(u W_gate^i) (.) u W_up^i) W_down^i) run over
+// the expert-sorted rows produced by dispatch (section "Алгоритм": each expert
+// receives all of its tokens in one call; an expert with no tokens is skipped).
+//
+// Two launches of one persistent, warp-specialised kernel:
+//   GEMM1 (kSwiGLU):  A = x_sorted [R, d],  B = W1[e] | W3[e]  ->  h = SiLU(a) (.) b, bf16
+//   GEMM2 (kDown):    A = h        [R, d_ff], B = W2[e]        ->  o (fp32)
+//
+// Tile: 128 rows (one TMEM lane per row) x 256 accumulator columns.  For GEMM1
+// the 256 columns are 128 columns of x W1 followed by the same 128 columns of
+// x W3, so the SwiGLU product is formed in the epilogue straight out of TMEM.
+// K advances 64 elements (one 128-byte swizzle row) per pipeline stage.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A box [128 x 64] (K-major) + B boxes [64 x 64] (MN-major)
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: tcgen05.ld -> SiLU(.) / convert -> global stores
+// Shared-memory stages are recycled through full/empty mbarriers; the two TMEM
+// accumulator buffers (2 x 256 columns) let the epilogue of tile i overlap the
+// MMAs of tile i+1.
+//
+// Weights stay in their natural row-major layout ([E, d, d_ff] and
+// [E, d_ff, d]); the B operand is read MN-major, which tcgen05 supports for
+// 16-bit types, so no repacking pass exists.
+//
+// Ragged groups: a tile starts at an expert's first row + 128*m and may run
+// past the expert's last row into the next expert's rows (or past R, where TMA
+// fills zeros); those rows are computed and discarded (stores are predicated).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "expert_gemm.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+namespace gemm {
+
+using namespace sm100;
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kBoxN = 64;
+constexpr int kMaxBoxes = 4;
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;                          // 16 KB
+constexpr int kBBoxBytes = kBK * kBoxN * 2;                     // 8 KB
+constexpr int kStageBytes = kABytes + kMaxBoxes * kBBoxBytes;   // 48 KB
+constexpr int kAccCols = 256;
+constexpr int kTmemCols = 2 * kAccCols;
+constexpr int kThreads = 192;
+constexpr int kMaxE = 32;
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024;
+
+struct Params {
+    const int32_t* offsets;  // [E+1]
+    void* out;               // GEMM1: bf16 h [R, n_out]; GEMM2: float o [R, n_out]
+    int* err;                // device status word
+    uint64_t timeout_ns;
+    int E;
+    int K;                   // contraction length
+    int n_out;               // output columns
+    int n_tile_out;          // output columns per tile
+    int n_boxes;             // B boxes per stage (MMA N = 64 * n_boxes)
+    int stall_after;         // test hook: producer stops after this many stages (-1: never)
+};
+
+struct TileInfo {
+    int e, row0, rows, n0;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int t, int E, const int* mt_prefix, const int* off,
+                                                int n_tiles, int n_tile_out) {
+    TileInfo ti;
+    int e = 0;
+    while (t >= n_tiles * mt_prefix[e + 1]) ++e;
+    const int local = t - n_tiles * mt_prefix[e];
+    const int mt = mt_prefix[e + 1] - mt_prefix[e];
+    const int n = local / mt;
+    const int m = local - n * mt;
+    ti.e = e;
+    ti.row0 = off[e] + m * kBM;
+    const int end = off[e + 1];
+    ti.rows = min(kBM, end - ti.row0);
+    ti.n0 = n * n_tile_out;
+    return ti;
+}
+
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB0,
+                       const __grid_constant__ CUtensorMap tmB1, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    __shared__ uint64_t full_bar[kStages];
+    __shared__ uint64_t empty_bar[kStages];
+    __shared__ uint64_t acc_full[2];
+    __shared__ uint64_t acc_empty[2];
+    __shared__ uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int s_off[kMaxE + 1];
+    __shared__ int s_mt[kMaxE + 1];
+    __shared__ volatile int s_abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(&drain_bar, 1);
+        fence_barrier_init();
+        s_abort = 0;
+        // m-tile prefix over experts (E <= 32, serial)
+        int acc = 0;
+        s_mt[0] = 0;
+        for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+        for (int e = 0; e < p.E; ++e) {
+            const int cnt = max(0, s_off[e + 1] - s_off[e]);
+            acc += (cnt + kBM - 1) / kBM;
+            s_mt[e + 1] = acc;
+        }
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB0);
+        if (kSwiGLU) tma_prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = tmem_slot;
+
+    const int n_tiles = p.n_out / p.n_tile_out;
+    const int total_tiles = s_mt[p.E] * n_tiles;
+    const int kb_count = p.K / kBK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_parity = 0;
+            int issued = 0;
+            bool ok = true;
+            const uint32_t tx_bytes = kABytes + p.n_boxes * kBBoxBytes;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                const TileInfo ti = decode_tile(t, p.E, s_mt, s_off, n_tiles, p.n_tile_out);
+                const int wrow0 = ti.e * p.K;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (p.stall_after >= 0 && issued >= p.stall_after) {
+                        ok = false;  // test hook: behave like a producer that died
+                        break;
+                    }
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns) || s_abort) {
+                        record_error(p.err, kDeviceTimeoutBase | kRoleProducer);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sA = smem + stage * kStageBytes;
+                    uint8_t* sB = sA + kABytes;
+                    mbar_arrive_expect_tx(&full_bar[stage], tx_bytes);
+                    tma_load_2d(sA, &tmA, &full_bar[stage], kb * kBK, ti.row0);
+                    const int wrow = wrow0 + kb * kBK;
+                    if (kSwiGLU) {
+                        tma_load_2d(sB, &tmB0, &full_bar[stage], ti.n0, wrow);
+                        tma_load_2d(sB + kBBoxBytes, &tmB0, &full_bar[stage], ti.n0 + kBoxN, wrow);
+                        tma_load_2d(sB + 2 * kBBoxBytes, &tmB1, &full_bar[stage], ti.n0, wrow);
+                        tma_load_2d(sB + 3 * kBBoxBytes, &tmB1, &full_bar[stage], ti.n0 + kBoxN,
+                                    wrow);
+                    } else {
+                        for (int j = 0; j < p.n_boxes; ++j)
+                            tma_load_2d(sB + j * kBBoxBytes, &tmB0, &full_bar[stage],
+                                        ti.n0 + j * kBoxN, wrow);
+                    }
+                    issued_mask |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) s_abort = 1;
+            // Every copy this thread issued must land before the CTA may exit.
+            for (int s = 0; s < kStages; ++s)
+                if (issued_mask & (1u << s))
+                    (void)mbar_wait(&full_bar[s], (issued_parity >> s) & 1u, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            const uint32_t idesc = idesc_bf16_f32(kBM, p.n_boxes * kBoxN, false, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns) || s_abort) {
+                    record_error(p.err, kDeviceTimeoutBase | kRoleMma);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kAccCols;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, p.timeout_ns) || s_abort) {
+                        record_error(p.err, kDeviceTimeoutBase | kRoleMma);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t adesc = desc_kmajor_sw128(a_addr + kk * 32);
+                        const uint64_t bdesc = desc_mnmajor_sw128(b_addr + kk * 2048, kBBoxBytes);
+                        tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0);
+                    }
+                    tc_commit(&empty_bar[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) s_abort = 1;
+            // Wait for every MMA this thread issued before TMEM is released.
+            tc_commit(&drain_bar);
+            (void)mbar_wait(&drain_bar, 0, p.timeout_ns);
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (warps 2..5)
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int row_in_tile = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+            const TileInfo ti = decode_tile(t, p.E, s_mt, s_off, n_tiles, p.n_tile_out);
+            const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
+            if (!got || s_abort) {
+                if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
+                s_abort = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t taddr = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
+            const bool valid = row_in_tile < ti.rows;
+            const int64_t grow = (int64_t)ti.row0 + row_in_tile;
+            if (kSwiGLU) {
+                __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                      grow * p.n_out + ti.n0;
+#pragma unroll 1
+                for (int c = 0; c < kAccCols / 2; c += 32) {
+                    uint32_t ra[32], rb[32];
+                    tmem_ld_32cols(taddr + c, ra);
+                    tmem_ld_32cols(taddr + kAccCols / 2 + c, rb);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float a0 = __uint_as_float(ra[2 * j]);
+                            const float a1 = __uint_as_float(ra[2 * j + 1]);
+                            const float b0 = __uint_as_float(rb[2 * j]);
+                            const float b1 = __uint_as_float(rb[2 * j + 1]);
+                            const float h0 = a0 / (1.0f + __expf(-a0)) * b0;
+                            const float h1 = a1 / (1.0f + __expf(-a1)) * b1;
+                            packed[j] = pack_bf16x2(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                                packed[4 * j + 3]);
+                    }
+                }
+            } else {
+                float* orow = reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0;
+                const int ncols = p.n_boxes * kBoxN;
+#pragma unroll 1
+                for (int c = 0; c < ncols; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32cols(taddr + c, r);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with a
+// [box_rows, 64]-element box and 128-byte swizzle.
+static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool kSwiGLU>
+static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                  const Params& p, int max_tiles, cudaStream_t stream) {
+    auto kern = expert_gemm_kernel<kSwiGLU>;
+    static int configured_device = -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (configured_device != dev) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytes) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        configured_device = dev;
+    }
+    const int grid = max(1, min(device_sm_count(), max_tiles));
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(a, b0, b1, p);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace gemm
+
+int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offsets, const void* W1,
+                 const void* W3, const void* W2, void* h, float* o, int* err,
+                 uint64_t timeout_ns, int stall_after, cudaStream_t stream,
+                 void* mid_event) {
+    using namespace gemm;
+    const int R = s.T * s.k;
+    if (R == 0) return MOE_OK;
+    CUtensorMap mx, mh, m1, m3, m2;
+    if (!make_map(&mx, x_sorted, (uint64_t)R, (uint64_t)s.d, kBM) ||
+        !make_map(&mh, h, (uint64_t)R, (uint64_t)s.d_ff, kBM) ||
+        !make_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
+        !make_map(&m3, W3, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
+        !make_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, kBK))
+        return MOE_ERR_CUDA;
+    // Upper bound on m-tiles: sum over experts of ceil(rows_e / 128).
+    const int max_mtiles = (R + kBM - 1) / kBM + s.E;
+
+    Params p1{};
+    p1.offsets = offsets;
+    p1.out = h;
+    p1.err = err;
+    p1.timeout_ns = timeout_ns;
+    p1.E = s.E;
+    p1.K = s.d;
+    p1.n_out = s.d_ff;
+    p1.n_tile_out = 128;
+    p1.n_boxes = 4;
+    p1.stall_after = stall_after;
+    int rc = launch<true>(mx, m1, m3, p1, max_mtiles * (s.d_ff / 128), stream);
+    if (rc != MOE_OK) return rc;
+    if (mid_event && cudaEventRecord(static_cast<cudaEvent_t>(mid_event), stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+
+    Params p2 = p1;
+    p2.out = o;
+    p2.K = s.d_ff;
+    p2.n_out = s.d;
+    p2.n_tile_out = (s.d % 256 == 0) ? 256 : 128;
+    p2.n_boxes = p2.n_tile_out / kBoxN;
+    p2.stall_after = -1;
+    return launch<false>(mh, m2, m2, p2, max_mtiles * (s.d / p2.n_tile_out), stream);
+}
+
+}  // namespace moe

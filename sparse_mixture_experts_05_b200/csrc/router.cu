@@ -1,0 +1,241 @@
+// router.cu -- router logits, top-k selection and softmax over the selected k.
+//
+// Mixtral textbook page, section "Прямой проход в формулах": g = u W_r,
+// S = TopK(g, k), w_i = exp(g_i) / sum_{j in S} exp(g_j); section "MoE изнутри":
+// the softmax runs over the k selected logits only, in float32.
+//
+// The contraction x[T,d] . Wg[d,E] is skinny (E = 8) and HBM-bound on reading
+// x once; it runs on mma.sync m16n8k16 (bf16 in, fp32 accumulate) so the issue
+// slots stay free for loads.  A warp owns 16 tokens and a quarter of d; the four
+// quarter sums are added in a fixed order, so results are deterministic.
+//
+// k-permutation: a dot product may pair its terms in any order, so a lane loads
+// 8 consecutive x elements (one 16-byte load) and feeds them to two MMAs as
+// fragment positions {2t,2t+1,2t+8,2t+9}; the router weights are staged in
+// shared memory in the matching order (one 16-byte load per lane per 32 k).
+//
+// Top-k: the four lanes of a quad hold the E logits of one token; k rounds of a
+// quad-shuffle argmax pick the largest logit not yet taken, lower expert index
+// first on ties (slot 0 = largest).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cfloat>
+#include <climits>
+
+#include "common.cuh"
+#include "router.cuh"
+
+namespace moe {
+namespace router {
+
+constexpr int kWarps = 16;
+constexpr int kKSplit = 4;
+constexpr int kSlots = kWarps / kKSplit;  // token tiles of 16 per block iteration
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxK = 8;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
+    return v > bv || (v == bv && id < bid) || bid == INT_MAX;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
+                  const float* __restrict__ bias, int T, int d, int E, int k,
+                  int32_t* __restrict__ idx, float* __restrict__ gate,
+                  float* __restrict__ logits) {
+    extern __shared__ uint4 s_wg[];  // [d/32][NT][32 lanes] x 8 bf16
+    __shared__ float s_red[kSlots][kKSplit][NT][32][4];
+
+    // Stage W_r in fragment order: entry (kb, nt, lane) holds
+    // Wg[kb*32 + (lane&3)*8 + j][nt*8 + (lane>>2)] for j = 0..7 (zero for n >= E).
+    const int nblk = d / 32;
+    for (int i = threadIdx.x; i < nblk * NT * 32; i += blockDim.x) {
+        const int ln = i & 31;
+        const int nt = (i >> 5) % NT;
+        const int kb = i / (32 * NT);
+        const int n = nt * 8 + (ln >> 2);
+        const int k0 = kb * 32 + (ln & 3) * 8;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = n < E ? wg[(int64_t)(k0 + 2 * j) * E + n] : 0u;
+            const uint32_t hi = n < E ? wg[(int64_t)(k0 + 2 * j + 1) * E + n] : 0u;
+            w[j] = lo | (hi << 16);
+        }
+        s_wg[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int slot = warp / kKSplit;
+    const int kq = warp % kKSplit;
+    const int g = lane >> 2;
+    const int t4 = lane & 3;
+    const int kper = d / kKSplit;
+    const int ntiles = (T + 15) / 16;
+
+    for (int base = blockIdx.x * kSlots; base < ntiles; base += gridDim.x * kSlots) {
+        const int tile = base + slot;
+        float c[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
+        if (tile < ntiles) {
+            const int r0 = tile * 16 + g;
+            const int r1 = r0 + 8;
+            const bool v0 = r0 < T, v1 = r1 < T;
+            const uint4* x0 = reinterpret_cast<const uint4*>(x + (int64_t)(v0 ? r0 : 0) * d);
+            const uint4* x1 = reinterpret_cast<const uint4*>(x + (int64_t)(v1 ? r1 : 0) * d);
+            const int kbeg = kq * kper, kend = kbeg + kper;
+#pragma unroll 4
+            for (int kb = kbeg; kb < kend; kb += 32) {
+                const int ci = (kb >> 3) + t4;
+                const uint4 a0 = v0 ? __ldg(x0 + ci) : make_uint4(0, 0, 0, 0);
+                const uint4 a1 = v1 ? __ldg(x1 + ci) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint4 b = s_wg[((kb >> 5) * NT + nt) * 32 + lane];
+                    mma_bf16_16816(c[nt], a0.x, a1.x, a0.y, a1.y, b.x, b.y);
+                    mma_bf16_16816(c[nt], a0.z, a1.z, a0.w, a1.w, b.z, b.w);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s_red[slot][kq][nt][lane][i] = c[nt][i];
+        }
+        __syncthreads();
+        if (kq == 0 && tile < ntiles) {
+            // v[nt][i]: token (i < 2 ? g : g+8), expert nt*8 + 2*t4 + (i & 1)
+            float v[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float sum = s_red[slot][0][nt][lane][i];
+                    sum = __fadd_rn(sum, s_red[slot][1][nt][lane][i]);
+                    sum = __fadd_rn(sum, s_red[slot][2][nt][lane][i]);
+                    sum = __fadd_rn(sum, s_red[slot][3][nt][lane][i]);
+                    const int n = nt * 8 + 2 * t4 + (i & 1);
+                    if (bias && n < E) sum = __fadd_rn(sum, bias[n]);
+                    v[nt][i] = sum;
+                }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int row = tile * 16 + g + 8 * half;
+                const bool rv = row < T;
+                if (logits && rv) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int n = nt * 8 + 2 * t4 + j;
+                            if (n < E) logits[(int64_t)row * E + n] = v[nt][2 * half + j];
+                        }
+                }
+                uint32_t taken = 0;  // bit (nt*2 + j) of this lane's candidates
+                float sel_v[kMaxK];
+                int sel_id[kMaxK];
+#pragma unroll
+                for (int s = 0; s < kMaxK; ++s) {
+                    if (s >= k) break;
+                    float bv = -FLT_MAX;
+                    int bid = INT_MAX;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int n = nt * 8 + 2 * t4 + j;
+                            const int bit = nt * 2 + j;
+                            const float cv = v[nt][2 * half + j];
+                            if (n < E && !(taken & (1u << bit)) && better(cv, n, bv, bid)) {
+                                bv = cv;
+                                bid = n;
+                            }
+                        }
+#pragma unroll
+                    for (int off = 1; off <= 2; off <<= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                        const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+                        if (oid != INT_MAX && better(ov, oid, bv, bid)) {
+                            bv = ov;
+                            bid = oid;
+                        }
+                    }
+                    // the lane that holds the winner marks it taken
+                    if (bid != INT_MAX && ((bid & 7) >> 1) == t4)
+                        taken |= 1u << ((bid >> 3) * 2 + (bid & 1));
+                    sel_v[s] = bv;
+                    sel_id[s] = bid;
+                }
+                if (rv && t4 == 0) {
+                    const float m = sel_v[0];
+                    float den = 0.f;
+                    float ex[kMaxK];
+#pragma unroll
+                    for (int s = 0; s < kMaxK; ++s) {
+                        if (s >= k) break;
+                        ex[s] = expf(sel_v[s] - m);
+                        den = __fadd_rn(den, ex[s]);
+                    }
+#pragma unroll
+                    for (int s = 0; s < kMaxK; ++s) {
+                        if (s >= k) break;
+                        idx[(int64_t)row * k + s] = sel_id[s];
+                        gate[(int64_t)row * k + s] = __fdiv_rn(ex[s], den);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace router
+
+int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
+                  int32_t* idx, float* gate, float* logits, cudaStream_t stream) {
+    using namespace router;
+    if (s.T == 0) return MOE_OK;
+    const int NT = (s.E + 7) / 8;
+    const size_t smem = (size_t)s.d * NT * 16;
+    const int ntiles = (s.T + 15) / 16;
+    const int grid = std::max(1, std::min(device_sm_count(), (ntiles + kSlots - 1) / kSlots));
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+    const uint16_t* wp = static_cast<const uint16_t*>(Wg);
+#define MOE_ROUTER_CASE(N)                                                                      \
+    case N: {                                                                                   \
+        auto kern = router_kernel<N>;                                                           \
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
+                                 (int)smem) != cudaSuccess)                                     \
+            return MOE_ERR_CUDA;                                                                \
+        kern<<<grid, kThreads, smem, stream>>>(xp, wp, bias, s.T, s.d, s.E, s.k, idx, gate,     \
+                                               logits);                                        \
+        break;                                                                                  \
+    }
+    switch (NT) {
+        MOE_ROUTER_CASE(1)
+        MOE_ROUTER_CASE(2)
+        MOE_ROUTER_CASE(3)
+        MOE_ROUTER_CASE(4)
+        default:
+            return MOE_ERR_UNSUPPORTED;
+    }
+#undef MOE_ROUTER_CASE
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

@@ -1,0 +1,88 @@
+"""Mixtral 8x7B shapes at full size (d = 4096, d_ff = 14336, E = 8, k = 2):
+prefill T = 4096, decode T = 16, skewed prefill T = 16384 with router bias.
+
+Routing is checked on every token; the expert kernel on sampled sorted rows
+(including the last row of every expert group, where tiles are ragged); the
+fused forward on sampled tokens through the oracle's per-token loop, and on
+every token for decode.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_mixture_experts_05_b200 as moe
+from sparse_mixture_experts_05_b200.inputs import workload_inputs
+
+from _parity import bf16_values, check_expert_rows, check_routing, check_y, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", params=["decode", "prefill", "skew"])
+def case(request):
+    inp = workload_inputs(request.param)
+    dev = to_dev(inp)
+    T, d, d_ff, E, k = inp["shape"]
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ws = moe.workspace(moe.moe_forward_workspace_bytes(inp["shape"]), "cuda")
+    y = moe.moe_forward(inp["shape"], dev["x"], dev["Wg"], dev["bias"], dev["W1"], dev["W3"],
+                        dev["W2"], idx_out=idx, gate_out=gate, ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    yield request.param, inp, dev, idx.cpu().numpy(), gate.cpu().numpy(), y
+    del dev, ws, y
+    torch.cuda.empty_cache()
+
+
+def test_routing_all_tokens(case):
+    name, inp, dev, g_idx, g_gate, y = case
+    T, d, d_ff, E, k = inp["shape"]
+    o_idx, o_gate, o_logits = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    _, stats = check_routing(g_idx, g_gate, o_idx, o_gate, o_logits, k)
+    print(name, stats)
+
+
+def test_forward_sampled_tokens(case):
+    name, inp, dev, g_idx, g_gate, y = case
+    T, d, d_ff, E, k = inp["shape"]
+    rng = np.random.default_rng(17)
+    toks = np.arange(T) if T <= 16 else np.unique(np.concatenate(
+        [[0, T - 1], rng.choice(T, 14, replace=False)]))
+    y_ref, r_idx, _ = oracle.forward_tokens(toks, inp["x"], inp["Wg"], inp["W1"], inp["W3"],
+                                            inp["W2"], k, bias=inp["bias"])
+    _, _, o_logits = oracle.route(inp["x"][torch.from_numpy(toks).long()], inp["Wg"], E, k,
+                                  bias=inp["bias"])
+    kth_tie, _ = oracle.near_tie_flags(o_logits, k)
+    same = np.array([set(g_idx[t]) == set(r_idx[i]) for i, t in enumerate(toks)])
+    assert np.all(same | kth_tie)
+    rows = same
+    yv = y[torch.from_numpy(toks).long().cuda()]
+    rel, ulps = check_y(yv, y_ref, rows=rows)
+    print(name, "max|y-y_ref|/rms", rel, "max ulps", ulps)
+
+
+def test_expert_sampled_rows(case):
+    name, inp, dev, g_idx, g_gate, y = case
+    T, d, d_ff, E, k = inp["shape"]
+    shape = inp["shape"]
+    offsets, perm, inv, xs = moe.moe_dispatch(shape, torch.from_numpy(g_idx).cuda(), dev["x"])
+    h, o, ws = moe.moe_expert_swiglu(shape, xs, offsets, dev["W1"], dev["W3"], dev["W2"])
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    off = offsets.cpu().numpy()
+    rng = np.random.default_rng(23)
+    rows = set()
+    for e in range(E):
+        if off[e + 1] > off[e]:
+            rows.update([int(off[e]), int(off[e + 1] - 1)])
+            rows.update(rng.integers(off[e], off[e + 1], 2).tolist())
+    rows = np.array(sorted(rows))
+    row_expert = np.searchsorted(off, rows, side="right") - 1
+    sub_off = np.concatenate([[0], np.cumsum(np.bincount(row_expert, minlength=E))]).astype(np.int32)
+    xs_sub = xs[torch.from_numpy(rows).long().cuda()].cpu()
+    h_ref, o_ref = oracle.expert(xs_sub, sub_off, inp["W1"], inp["W3"], inp["W2"])
+    sel = torch.from_numpy(rows).long().cuda()
+    frac, worst = check_expert_rows(bf16_values(h[sel]), o[sel].cpu().numpy().astype(np.float64),
+                                    bf16_values(xs_sub), row_expert, inp["W1"], inp["W3"],
+                                    inp["W2"], h_ref, o_ref)
+    print(name, "h elements differing from the oracle", frac, "o error / bound", worst)

@@ -1,0 +1,249 @@
+"""CUDA path vs CPU oracle, element by element, through the C ABI.
+
+Every kernel is checked on its own (same inputs on both sides) and the fused
+forward is checked end to end, on the tiny and quarter-width workloads, on
+ragged and degenerate shapes, and -- in test_gpu_fullsize.py -- on the
+Mixtral 8x7B workloads at full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_mixture_experts_05_b200 as moe
+from sparse_mixture_experts_05_b200.inputs import identical_experts, make_inputs, workload_inputs
+
+from _parity import (bf16_ulp, bf16_values, check_expert_rows, check_routing, check_y, to_dev,
+                     u16)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # name: (T, d, d_ff, E, k, seed, bias)
+    "tiny": (64, 128, 256, 8, 2, 0, False),
+    "ragged": (77, 256, 384, 8, 2, 5, False),
+    "tail": (300, 128, 256, 8, 2, 6, True),
+    "k1": (50, 128, 256, 8, 1, 7, False),
+    "E1k1": (40, 128, 128, 1, 1, 8, False),
+    "E16k4": (96, 256, 256, 16, 4, 9, False),
+    "E5k3": (33, 128, 256, 5, 3, 10, False),
+    "single": (1, 128, 256, 8, 2, 11, False),
+}
+
+
+def _inputs(name):
+    if name == "quarter":
+        return workload_inputs("quarter")
+    T, d, d_ff, E, k, seed, bias = CASES[name]
+    return make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+
+
+ALL = list(CASES) + ["quarter"]
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_route(name):
+    inp = _inputs(name)
+    T, d, d_ff, E, k = inp["shape"]
+    dev = to_dev(inp)
+    idx, gate, logits = moe.moe_route(inp["shape"], dev["x"], dev["Wg"], dev["bias"],
+                                      want_logits=True)
+    torch.cuda.synchronize()
+    o_idx, o_gate, o_logits = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    lerr = np.max(np.abs(logits.cpu().numpy() - o_logits))
+    assert lerr < 1e-4, lerr
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), o_idx, o_gate, o_logits, k)
+
+
+def test_route_ties_to_lower_index():
+    inp = make_inputs(48, 128, 256, 8, 2, seed=12)
+    inp["Wg"][:, 6] = inp["Wg"][:, 3]
+    inp["x"][:, 0] = 1.0
+    inp["Wg"][0, 3] = inp["Wg"][0, 6] = 40.0
+    dev = to_dev(inp)
+    idx, gate, logits = moe.moe_route(inp["shape"], dev["x"], dev["Wg"], want_logits=True)
+    idx = idx.cpu().numpy()
+    lg = logits.cpu().numpy()
+    assert np.all(lg[:, 3] == lg[:, 6])
+    assert np.all(idx[:, 0] == 3) and np.all(idx[:, 1] == 6)
+    assert np.all(gate.cpu().numpy() == 0.5)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_dispatch_bit_exact(name):
+    inp = _inputs(name)
+    T, d, d_ff, E, k = inp["shape"]
+    o_idx, _, _ = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    dev = to_dev(inp)
+    offsets, perm, inv, xs = moe.moe_dispatch(inp["shape"], torch.from_numpy(o_idx).cuda(),
+                                              dev["x"])
+    r_off, r_perm, r_inv = oracle.dispatch(o_idx, E)
+    assert np.array_equal(offsets.cpu().numpy(), r_off)
+    assert np.array_equal(perm.cpu().numpy(), r_perm)
+    assert np.array_equal(inv.cpu().numpy(), r_inv)
+    assert np.array_equal(u16(xs), oracle.gather(inp["x"], r_perm))
+
+
+def test_dispatch_skips_out_of_range_ids():
+    T, d, E, k = 40, 128, 8, 2
+    x = torch.randn(T, d).to(torch.bfloat16).cuda()
+    idx = torch.randint(0, E, (T, k), dtype=torch.int32)
+    idx[:, 1] = (idx[:, 0] + 1) % E
+    idx[5, 1] = -1
+    idx[9, 0] = E
+    offsets, perm, inv, xs = moe.moe_dispatch((T, d, 256, E, k), idx.cuda(), x)
+    inv = inv.cpu().numpy()
+    assert inv[5, 1] == -1 and inv[9, 0] == -1
+    assert offsets.cpu().numpy()[-1] == T * k - 2
+    valid = idx.numpy()
+    keep = (valid >= 0) & (valid < E)
+    assert np.all(inv[keep] >= 0)
+    assert np.array_equal(np.sort(inv[keep]), np.arange(T * k - 2))
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_expert_swiglu(name):
+    inp = _inputs(name)
+    T, d, d_ff, E, k = inp["shape"]
+    o_idx, _, _ = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    r_off, r_perm, _ = oracle.dispatch(o_idx, E)
+    xs = oracle.gather(inp["x"], r_perm)
+    h_ref, o_ref = oracle.expert(xs, r_off, inp["W1"], inp["W3"], inp["W2"])
+    dev = to_dev(inp)
+    xs_t = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16).cuda()
+    h, o, ws = moe.moe_expert_swiglu(inp["shape"], xs_t, torch.from_numpy(r_off).cuda(),
+                                     dev["W1"], dev["W3"], dev["W2"])
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    row_expert = np.searchsorted(r_off, np.arange(T * k), side="right") - 1
+    check_expert_rows(bf16_values(h), o.cpu().numpy().astype(np.float64), oracle.bf16_to_f64(xs),
+                      row_expert, inp["W1"], inp["W3"], inp["W2"], h_ref, o_ref)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_combine(name):
+    inp = _inputs(name)
+    T, d, d_ff, E, k = inp["shape"]
+    rng = np.random.default_rng(3)
+    o32 = rng.standard_normal((T * k, d)).astype(np.float32)
+    inv = rng.permutation(T * k).reshape(T, k).astype(np.int32)
+    gate = rng.random((T, k)).astype(np.float32)
+    gate /= gate.sum(1, keepdims=True)
+    y = moe.moe_combine(inp["shape"], torch.from_numpy(o32).cuda(), torch.from_numpy(inv).cuda(),
+                        torch.from_numpy(gate).cuda())
+    y_ref = oracle.combine(o32.astype(np.float64), inv, gate)
+    err = np.abs(bf16_values(y) - y_ref)
+    # float32 products and their sum each round once (relative 2^-24 of their own
+    # magnitude), then y rounds once to bf16: |err| <= ulp/2 + 2^-23 * sum_s |g_s o_s|
+    mag = oracle.combine(np.abs(o32.astype(np.float64)), inv, gate)
+    assert np.all(err <= 0.5 * bf16_ulp(y_ref) + 2.0 ** -23 * mag + 1e-30)
+    assert np.mean(err > 0.5 * bf16_ulp(y_ref)) < 1e-3
+
+
+def _forward_and_check(inp, ws=None):
+    T, d, d_ff, E, k = inp["shape"]
+    dev = to_dev(inp)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    y = moe.moe_forward(inp["shape"], dev["x"], dev["Wg"], dev["bias"], dev["W1"], dev["W3"],
+                        dev["W2"], idx_out=idx, gate_out=gate, ws=ws)
+    torch.cuda.synchronize()
+    o_idx, o_gate, o_logits = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    g_idx = idx.cpu().numpy()
+    g_gate = gate.cpu().numpy()
+    strict, stats = check_routing(g_idx, g_gate, o_idx, o_gate, o_logits, k)
+    y_ref, _, _ = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k,
+                                 bias=inp["bias"])
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    rel, ulps = check_y(y, y_ref, rows=strict, rms_ref=rms)
+    # forced routing: the GPU's idx/gate through the oracle's dispatch, experts and combine
+    if not np.all(strict):
+        f_off, f_perm, f_inv = oracle.dispatch(g_idx, E)
+        _, f_o = oracle.expert(oracle.gather(inp["x"], f_perm), f_off, inp["W1"], inp["W3"],
+                               inp["W2"])
+        y_forced = oracle.combine(f_o, f_inv, g_gate)
+        check_y(y, y_forced, rows=~strict, rms_ref=rms)
+    return y, stats, rel
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_forward(name):
+    _forward_and_check(_inputs(name))
+
+
+def test_forward_identical_experts_equal_swiglu():
+    inp = identical_experts(make_inputs(64, 128, 256, 8, 2, seed=13))
+    y, _, _ = _forward_and_check(inp)
+    x = bf16_values(inp["x"])
+    W1 = bf16_values(inp["W1"][0])
+    W3 = bf16_values(inp["W3"][0])
+    W2 = bf16_values(inp["W2"][0])
+    a = x @ W1
+    ref = ((a / (1 + np.exp(-a))) * (x @ W3)) @ W2
+    assert np.max(np.abs(bf16_values(y) - ref)) <= 2e-2 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_forward_all_tokens_one_expert():
+    inp = make_inputs(200, 128, 256, 8, 2, seed=14)
+    inp["bias"] = torch.tensor([0, 0, 0, 50.0, 0, 0, 0, 0], dtype=torch.float32)
+    y, _, _ = _forward_and_check(inp)
+
+
+def test_forward_empty_batch_is_noop():
+    inp = make_inputs(0, 128, 256, 8, 2, seed=15)
+    dev = to_dev(inp)
+    y = torch.full((0, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward(inp["shape"], dev["x"], dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"], y=y,
+                    ws=moe.workspace(4096, "cuda"))
+    torch.cuda.synchronize()
+
+
+def test_forward_deterministic_and_hostio_matches():
+    inp = workload_inputs("tiny")
+    T, d, d_ff, E, k = inp["shape"]
+    dev = to_dev(inp)
+    ws = moe.workspace(moe.moe_forward_hostio_workspace_bytes(inp["shape"]), "cuda")
+    y1 = moe.moe_forward(inp["shape"], dev["x"], dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"],
+                         ws=ws)
+    y2 = moe.moe_forward(inp["shape"], dev["x"], dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"],
+                         ws=ws)
+    x_host = inp["x"].clone().pin_memory()
+    y_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    moe.moe_forward_hostio(inp["shape"], x_host, dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"],
+                           y_host, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert torch.equal(y1.cpu(), y_host)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    inp = workload_inputs("tiny")
+    T, d, d_ff, E, k = inp["shape"]
+    o_idx, _, _ = oracle.route(inp["x"], inp["Wg"], E, k)
+    r_off, r_perm, _ = oracle.dispatch(o_idx, E)
+    xs = torch.from_numpy(oracle.gather(inp["x"], r_perm).view(np.int16)).view(torch.bfloat16).cuda()
+    dev = to_dev(inp)
+    off = torch.from_numpy(r_off).cuda()
+    _, _, ws = moe.moe_expert_swiglu_stall_test(inp["shape"], xs, off, dev["W1"], dev["W3"],
+                                                dev["W2"], stall_after=1, timeout_ns=2_000_000)
+    assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    # the context is still usable and the next call clears the status word
+    h, o, ws = moe.moe_expert_swiglu(inp["shape"], xs, off, dev["W1"], dev["W3"], dev["W2"], ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    xs_np = oracle.gather(inp["x"], r_perm)
+    h_ref, o_ref = oracle.expert(xs_np, r_off, inp["W1"], inp["W3"], inp["W2"])
+    row_expert = np.searchsorted(r_off, np.arange(T * k), side="right") - 1
+    check_expert_rows(bf16_values(h), o.cpu().numpy().astype(np.float64), oracle.bf16_to_f64(xs_np),
+                      row_expert, inp["W1"], inp["W3"], inp["W2"], h_ref, o_ref)
+
+
+def test_host_checks_launch_nothing():
+    inp = workload_inputs("tiny")
+    dev = to_dev(inp)
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_route((64, 128, 256, 8, 9), dev["x"], torch.empty(128, 8, dtype=torch.bfloat16,
+                                                                  device="cuda"))
+    assert e.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_forward(inp["shape"], dev["x"], dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"],
+                        ws=moe.workspace(1024, "cuda"))
+    assert e.value.status == moe.MOE_ERR_WORKSPACE
