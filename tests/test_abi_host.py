@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/moe.h declares, and rejects bad arguments before it
+touches the device (the counterpart of the ValueError the Mixtral textbook
+page's MoE constructor raises for top_k_experts outside 1..num_experts,
+sections "Mixtral" and "Конфигурация")."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_05_b200 as moe
+from sparse_mixture_experts_05_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    declared = _declared()
+    assert declared, "no declarations found"
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(binding.EXPORTS)
+
+
+def test_status_strings():
+    for code in range(6):
+        assert binding.status_string(code).startswith("MOE_")
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((64, 128, 256, 8, 2), moe.MOE_OK),
+    ((0, 128, 256, 8, 2), moe.MOE_OK),
+    ((64, 128, 256, 8, 0), moe.MOE_ERR_INVALID_ARG),   # k outside 1..E
+    ((64, 128, 256, 8, 9), moe.MOE_ERR_INVALID_ARG),
+    ((-1, 128, 256, 8, 2), moe.MOE_ERR_INVALID_ARG),
+    ((64, 100, 256, 8, 2), moe.MOE_ERR_UNSUPPORTED),   # d not a multiple of 128
+    ((64, 128, 200, 8, 2), moe.MOE_ERR_UNSUPPORTED),
+    ((64, 128, 256, 33, 2), moe.MOE_ERR_UNSUPPORTED),  # E > 32
+    ((64, 128, 256, 16, 9), moe.MOE_ERR_UNSUPPORTED),  # k > 8
+    ((16, 4096, 14336, 32, 2), moe.MOE_ERR_UNSUPPORTED),  # router tile too large
+    ((1 << 20, 4096, 14336, 8, 2), moe.MOE_ERR_UNSUPPORTED),  # 32-bit row index overflow
+])
+def test_shape_checks(shape, code):
+    assert moe.moe_check_shape(shape) == code
+
+
+def test_workspace_sizes():
+    s = (4096, 4096, 14336, 8, 2)
+    fwd = moe.moe_forward_workspace_bytes(s)
+    R = 4096 * 2
+    assert fwd >= R * 4096 * 2 + R * 14336 * 2 + R * 4096 * 4
+    assert moe.moe_forward_hostio_workspace_bytes(s) == fwd + 2 * 4096 * 4096 * 2
+    assert moe.moe_expert_workspace_bytes(s) >= 4
+    assert moe.moe_forward_workspace_bytes((64, 128, 256, 8, 9)) == 0
+
+
+def _call(fn, *args):
+    return getattr(binding.lib(), fn)(*args)
+
+
+def test_null_and_misaligned_pointers_are_rejected_without_launch():
+    S = binding.MoeShape(64, 128, 256, 8, 2)
+    P = ctypes.c_void_p
+    good = P(1 << 20)          # never dereferenced: validation fails first
+    bad = P((1 << 20) + 8)     # not 16-byte aligned
+    assert _call("moe_route", S, None, good, None, good, good, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_route", S, bad, good, None, good, good, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_combine", S, good, None, good, good, None) == moe.MOE_ERR_INVALID_ARG
+    # every call below carries one invalid argument, so nothing may reach the device
+    assert _call("moe_expert_swiglu", S, good, good, good, good, good, None, good, good,
+                 ctypes.c_size_t(1 << 20), None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_expert_swiglu", S, good, good, good, good, good, good, good, good,
+                 ctypes.c_size_t(16), None) == moe.MOE_ERR_WORKSPACE
+    assert _call("moe_forward", S, good, good, None, good, good, good, good, None, None, good,
+                 ctypes.c_size_t(16), None) == moe.MOE_ERR_WORKSPACE
+    bad_k = binding.MoeShape(64, 128, 256, 8, 9)
+    assert _call("moe_forward", bad_k, good, good, None, good, good, good, good, None, None, good,
+                 ctypes.c_size_t(1 << 30), None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_forward_profiled", S, good, good, None, good, good, good, good, good,
+                 ctypes.c_size_t(1 << 30), None, 7, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_expert_swiglu_stall_test", S, good, good, good, good, good, good, good,
+                 good, ctypes.c_size_t(1 << 20), -1, ctypes.c_uint64(10 ** 6),
+                 None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op_on_host():
+    S = binding.MoeShape(0, 128, 256, 8, 2)
+    for fn, nargs in (("moe_route", 7), ("moe_combine", 5)):
+        assert _call(fn, S, *([None] * nargs)) == moe.MOE_OK
