@@ -185,6 +185,37 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
                        size_t ws_bytes, void* stream);
 
 /*
+ * moe_forward_static -- moe_forward for callers that cannot allocate device
+ * memory.  No counterpart on the pages: it exists for callers such as code
+ * running while a stream is being captured into a CUDA graph (where cudaMalloc
+ * is not allowed), plugins that run inside a host framework which owns every
+ * allocation and hands out none, and latency-critical serving loops that must
+ * not hit cudaMalloc's implicit device synchronisation.  Instead of a
+ * caller-provided workspace it uses a fixed scratch array of 8 MiB
+ * (MOE_STATIC_SCRATCH_BYTES) in device memory, compiled into the library; every
+ * GPU on which the library is loaded reserves it until the process exits.  The
+ * caller still passes every input and the output y, all in device memory.
+ *  - Limit: shapes with moe_forward_workspace_bytes(s) > 8 MiB are rejected
+ *    with MOE_ERR_WORKSPACE before anything is launched (for d = 4096,
+ *    d_ff = 14336, k = 2 that allows T <= 64 tokens: decode-sized batches).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture begins.
+ *  - Calls share the one array and it keeps the previous call's contents; the
+ *    call clears the part that must start at zero (its status word) itself.
+ *    Calls whose work overlaps on the GPU (different streams, or different
+ *    host threads, on one device) race on the array: serialise them.
+ *  - device_status: nullable device int32; when given, it receives the call's
+ *    status word (0, or nonzero after an expired device wait; see
+ *    moe_read_device_status) once the call's work has run.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define MOE_STATIC_SCRATCH_BYTES (8u << 20)
+int moe_forward_static(moe_shape s, const void* x, const void* Wg, const float* bias,
+                       const void* W1, const void* W3, const void* W2, void* y,
+                       int32_t* device_status, void* stream);
+
+/*
  * moe_read_device_status -- SYNCHRONISES `stream`, then reads the status word
  * that moe_expert_swiglu / moe_forward keep at the start of their workspace:
  * MOE_OK, or MOE_ERR_DEVICE_TIMEOUT when a bounded device wait gave up

@@ -29,8 +29,11 @@ EXPORTS = (
     "moe_status_string", "moe_check_shape", "moe_expert_workspace_bytes",
     "moe_forward_workspace_bytes", "moe_forward_hostio_workspace_bytes", "moe_route",
     "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_stall_test", "moe_combine",
-    "moe_forward", "moe_forward_profiled", "moe_forward_hostio", "moe_read_device_status",
+    "moe_forward", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_static",
+    "moe_read_device_status",
 )
+
+MOE_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class MoeShape(ctypes.Structure):
@@ -84,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, Z, P, I, P]
         L.moe_forward_hostio.restype = I
         L.moe_forward_hostio.argtypes = [S, P, P, P, P, P, P, P, P, Z, P]
+        L.moe_forward_static.restype = I
+        L.moe_forward_static.argtypes = [S, P, P, P, P, P, P, P, P, P]
         L.moe_read_device_status.restype = I
         L.moe_read_device_status.argtypes = [P, P]
         _lib = L
@@ -305,6 +310,27 @@ def moe_forward_hostio(shape, x_host, Wg, bias, W1, W3, W2, y_host, ws, stream=N
            lib().moe_forward_hostio(_shape(shape), _p(x_host), _p(Wg), _p(bias), _p(W1), _p(W3),
                                     _p(W2), _p(y_host), _p(ws), ws.numel(), _stream(stream)))
     return y_host
+
+
+def moe_forward_static(shape, x, Wg, bias, W1, W3, W2, y=None, device_status=None, stream=None):
+    """moe_forward without a workspace argument: the library's fixed 8 MiB device
+    scratch array stands in for it (for callers that cannot allocate device memory).
+    `device_status`: optional CUDA int32 tensor of one element that receives the
+    call's status word."""
+    T, d, d_ff, E, k = shape
+    _dev(x, "x", torch.bfloat16, (T, d))
+    _dev(Wg, "Wg", torch.bfloat16, (d, E))
+    _dev(bias, "bias", torch.float32, (E,))
+    _dev(W1, "W1", torch.bfloat16, (E, d, d_ff))
+    _dev(W3, "W3", torch.bfloat16, (E, d, d_ff))
+    _dev(W2, "W2", torch.bfloat16, (E, d_ff, d))
+    y = _new((T, d), torch.bfloat16, x) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, d))
+    _dev(device_status, "device_status", torch.int32, (1,))
+    _check("moe_forward_static",
+           lib().moe_forward_static(_shape(shape), _p(x), _p(Wg), _p(bias), _p(W1), _p(W3),
+                                    _p(W2), _p(y), _p(device_status), _stream(stream)))
+    return y
 
 
 def moe_read_device_status(ws, stream=None) -> int:

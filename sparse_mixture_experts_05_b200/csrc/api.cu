@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "combine.cuh"
 #include "common.cuh"
@@ -120,6 +121,29 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     rc = launch_combine(s, o, inv, gate, y, st);
     if (rc) return rc;
     return mark(6) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Scratch of moe_forward_static: a fixed 8 MiB array in device memory that
+// every GPU which loads this library holds until the process exits.  Host code
+// only ever sees a host-side stand-in for this name; the device address comes
+// from cudaGetSymbolAddress, once per device.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device (looked up on the
+// first call per device, with that device current).  nullptr on failure.
+void* static_scratch_address() {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
 }
 
 }  // namespace
@@ -270,6 +294,29 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
     rc = forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st, nullptr);
     if (rc) return rc;
     if (cudaMemcpyAsync(y_host, y_dev, io_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int moe_forward_static(moe_shape s, const void* x, const void* Wg, const float* bias,
+                       const void* W1, const void* W3, const void* W2, void* y,
+                       int32_t* device_status, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(y) || !ok_opt(device_status))
+        return MOE_ERR_INVALID_ARG;
+    if (moe_forward_workspace_bytes(s) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+    void* ws = static_scratch_address();
+    if (!ws) return MOE_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // forward_impl zeroes the status word (first word of the scratch) itself and
+    // overwrites every other scratch byte it reads, so nothing else needs clearing.
+    rc = forward_impl(s, x, Wg, bias, W1, W3, W2, y, nullptr, nullptr, ws, st, nullptr);
+    if (rc) return rc;
+    if (device_status &&
+        cudaMemcpyAsync(device_status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+            cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -64,6 +64,9 @@ def test_workspace_sizes():
     assert moe.moe_forward_hostio_workspace_bytes(s) == fwd + 2 * 4096 * 4096 * 2
     assert moe.moe_expert_workspace_bytes(s) >= 4
     assert moe.moe_forward_workspace_bytes((64, 128, 256, 8, 9)) == 0
+    # decode batches of the Mixtral shape fit the static scratch, larger ones do not
+    assert moe.moe_forward_workspace_bytes((64, 4096, 14336, 8, 2)) <= binding.MOE_STATIC_SCRATCH_BYTES
+    assert moe.moe_forward_workspace_bytes((80, 4096, 14336, 8, 2)) > binding.MOE_STATIC_SCRATCH_BYTES
 
 
 def _call(fn, *args):
@@ -88,6 +91,10 @@ def test_null_and_misaligned_pointers_are_rejected_without_launch():
     bad_k = binding.MoeShape(64, 128, 256, 8, 9)
     assert _call("moe_forward", bad_k, good, good, None, good, good, good, good, None, None, good,
                  ctypes.c_size_t(1 << 30), None) == moe.MOE_ERR_INVALID_ARG
+    big = (1024, 1024, 3584, 8, 2)
+    assert moe.moe_forward_workspace_bytes(big) > binding.MOE_STATIC_SCRATCH_BYTES
+    assert _call("moe_forward_static", binding.MoeShape(*big), good, good, None,
+                 good, good, good, good, None, None) == moe.MOE_ERR_WORKSPACE
     assert _call("moe_forward_profiled", S, good, good, None, good, good, good, good, good,
                  ctypes.c_size_t(1 << 30), None, 7, None) == moe.MOE_ERR_INVALID_ARG
     assert _call("moe_expert_swiglu_stall_test", S, good, good, good, good, good, good, good,
