@@ -59,6 +59,10 @@ def parse(argv=None):
                     help="skip the decode-workload line added to the prefill run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (smaller cases for profiler captures)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (smaller cases for profiler captures)")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -209,13 +213,33 @@ def algorithmic(shape, counts):
     }
 
 
-def time_workload(name, steps, warmup, device, rank):
+def workload(name, tokens=None, experts=None):
+    import dataclasses
+
+    from sparse_mixture_experts_05_b200.inputs import WORKLOADS
+    w = WORKLOADS[name]
+    if tokens is not None:
+        w = dataclasses.replace(w, T=tokens)
+    if experts is not None:
+        w = dataclasses.replace(w, E=experts)
+    return w
+
+
+def workload_label(a):
+    label = WORKLOAD_NAMES[a.workload]
+    if a.tokens is not None or a.experts is not None:
+        w = workload(a.workload, a.tokens, a.experts)
+        label += f" (profiling override: T={w.T} E={w.E})"
+    return label
+
+
+def time_workload(name, steps, warmup, device, rank, tokens=None, experts=None):
     import torch
 
     import sparse_mixture_experts_05_b200 as moe
-    from sparse_mixture_experts_05_b200.inputs import WORKLOADS, make_inputs
+    from sparse_mixture_experts_05_b200.inputs import make_inputs
 
-    w = WORKLOADS[name]
+    w = workload(name, tokens, experts)
     inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
     shape = inp["shape"]
     x, Wg, bias, W1, W3, W2 = (inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
@@ -337,7 +361,7 @@ def run_ours(a):
     peaks, peak_kind = load_peaks()
     moe.binding.lib()
 
-    ctx = time_workload(a.workload, a.steps, a.warmup, device, rank)
+    ctx = time_workload(a.workload, a.steps, a.warmup, device, rank, a.tokens, a.experts)
     clock = ClockSampler(local)
     step_ms, parts, bracket_ms, clocks = timed_loop(ctx, a.steps, pg, device, clock)
     mean_ms = statistics.mean(step_ms)
@@ -378,7 +402,7 @@ def run_ours(a):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) tokens and N(0,1/fan_in) bf16 weights (no dataset, "
                 "no trained weights)",
-        "config": {"workload": WORKLOAD_NAMES[a.workload], "model": "Mixtral 8x7B MoE layer",
+        "config": {"workload": workload_label(a), "model": "Mixtral 8x7B MoE layer",
                    "T": T, "d": shape[1], "d_ff": shape[2], "E": shape[3], "k": shape[4],
                    "global_batch": T * world, "seq_len": T, "parallelism": f"replicas x{world}",
                    "l2": "flushed: 512 MiB written between timed steps (flush not timed)",
@@ -396,7 +420,7 @@ def run_ours(a):
     del ctx
     torch.cuda.empty_cache()
 
-    if a.workload == "prefill" and not a.no_secondary:
+    if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
         dctx = time_workload("decode", a.steps, a.warmup, device, rank)
         d_ms, d_parts, _, d_clocks = timed_loop(dctx, a.steps, pg, device, ClockSampler(local))
         d_mean = reduce_max(pg, statistics.mean(d_ms), device)
@@ -412,14 +436,12 @@ def run_ours(a):
                                (d_mean / 1000) / 1e9, 1),
             "kernel_ms": {k_: round(v, 4) for k_, v in d_parts.items()},
             "expert_rows": dctx["counts"], "clocks": d_clocks}
-        if world == 1 and rank == 0 and not a.no_cpu_baseline:
-            pass
         del dctx
         torch.cuda.empty_cache()
 
     if world == 1 and rank == 0 and not a.no_cpu_baseline:
-        from sparse_mixture_experts_05_b200.inputs import WORKLOADS, make_inputs
-        w = WORKLOADS[a.workload]
+        from sparse_mixture_experts_05_b200.inputs import make_inputs
+        w = workload(a.workload, a.tokens, a.experts)
         inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
         cb, _ = oracle_sample(inp, a.cpu_seconds)
         line["cpu_baseline"] = cb
@@ -436,11 +458,11 @@ def run_reference(a):
         return
     import torch
 
-    from sparse_mixture_experts_05_b200.inputs import WORKLOADS, make_inputs
     import numpy as np
 
     import oracle
-    w = WORKLOADS[a.workload]
+    from sparse_mixture_experts_05_b200.inputs import make_inputs
+    w = workload(a.workload, a.tokens, a.experts)
     device = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
     host = {key: (inp[key].cpu() if inp[key] is not None else None)
@@ -472,7 +494,7 @@ def run_reference(a):
         "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": round(step_s * 1000, 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe and seeds)",
-        "config": {"workload": WORKLOAD_NAMES[a.workload], "model": "Mixtral 8x7B MoE layer",
+        "config": {"workload": workload_label(a), "model": "Mixtral 8x7B MoE layer",
                    "T": T, "d": w.d, "d_ff": w.d_ff, "E": w.E, "k": w.k,
                    "global_batch": T, "seq_len": T, "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,

@@ -76,8 +76,11 @@ struct TileInfo {
     int e, row0, rows, n0;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(int t, int E, const int* mt_prefix, const int* off,
-                                                int n_tiles, int n_tile_out) {
+// Tile t of the expert-major enumeration: expert e owns tiles
+// [n_tiles * mt_prefix[e], n_tiles * mt_prefix[e+1]), n-major within an
+// expert with m fastest, so tiles that run at the same time share weight tiles.
+__device__ __forceinline__ TileInfo decode_tile_rows(int t, const int* mt_prefix, const int* off,
+                                                     int n_tiles, int n_tile_out, int tile_rows) {
     TileInfo ti;
     int e = 0;
     while (t >= n_tiles * mt_prefix[e + 1]) ++e;
@@ -86,11 +89,57 @@ __device__ __forceinline__ TileInfo decode_tile(int t, int E, const int* mt_pref
     const int n = local / mt;
     const int m = local - n * mt;
     ti.e = e;
-    ti.row0 = off[e] + m * kBM;
-    const int end = off[e + 1];
-    ti.rows = min(kBM, end - ti.row0);
+    ti.row0 = off[e] + m * tile_rows;
+    ti.rows = min(tile_rows, off[e + 1] - ti.row0);
     ti.n0 = n * n_tile_out;
     return ti;
+}
+
+// GEMM1 epilogue of one TMEM lane (= one row): columns [0,128) hold a = x W1,
+// columns [128,256) hold b = x W3; h = SiLU(a) * b = a / (1 + exp(-a)) * b.
+__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, __nv_bfloat16* hrow) {
+#pragma unroll 1
+    for (int c = 0; c < kAccCols / 2; c += 32) {
+        uint32_t ra[32], rb[32];
+        tmem_ld_32cols(taddr + c, ra);
+        tmem_ld_32cols(taddr + kAccCols / 2 + c, rb);
+        tmem_ld_wait();
+        if (valid) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float a0 = __uint_as_float(ra[2 * j]);
+                const float a1 = __uint_as_float(ra[2 * j + 1]);
+                const float b0 = __uint_as_float(rb[2 * j]);
+                const float b1 = __uint_as_float(rb[2 * j + 1]);
+                const float h0 = a0 / (1.0f + __expf(-a0)) * b0;
+                const float h1 = a1 / (1.0f + __expf(-a1)) * b1;
+                packed[j] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                    packed[4 * j + 3]);
+        }
+    }
+}
+
+// GEMM2 epilogue of one TMEM lane: `ncols` fp32 columns stored as they are.
+__device__ __forceinline__ void epilogue_store_f32(uint32_t taddr, bool valid, float* orow,
+                                                   int ncols) {
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32cols(taddr + c, r);
+        tmem_ld_wait();
+        if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                dst[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        }
+    }
 }
 
 template <bool kSwiGLU>
@@ -165,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             const uint32_t tx_bytes = kABytes + p.n_boxes * kBBoxBytes;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = decode_tile(t, p.E, s_mt, s_off, n_tiles, p.n_tile_out);
+                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM);
                 const int wrow0 = ti.e * p.K;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (p.stall_after >= 0 && issued >= p.stall_after) {
@@ -263,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-            const TileInfo ti = decode_tile(t, p.E, s_mt, s_off, n_tiles, p.n_tile_out);
+            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
                 if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
@@ -274,50 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t taddr = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
             const bool valid = row_in_tile < ti.rows;
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
-            if (kSwiGLU) {
-                __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                      grow * p.n_out + ti.n0;
-#pragma unroll 1
-                for (int c = 0; c < kAccCols / 2; c += 32) {
-                    uint32_t ra[32], rb[32];
-                    tmem_ld_32cols(taddr + c, ra);
-                    tmem_ld_32cols(taddr + kAccCols / 2 + c, rb);
-                    tmem_ld_wait();
-                    if (valid) {
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float a0 = __uint_as_float(ra[2 * j]);
-                            const float a1 = __uint_as_float(ra[2 * j + 1]);
-                            const float b0 = __uint_as_float(rb[2 * j]);
-                            const float b1 = __uint_as_float(rb[2 * j + 1]);
-                            const float h0 = a0 / (1.0f + __expf(-a0)) * b0;
-                            const float h1 = a1 / (1.0f + __expf(-a1)) * b1;
-                            packed[j] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(hrow + c);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                                packed[4 * j + 3]);
-                    }
-                }
-            } else {
-                float* orow = reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0;
-                const int ncols = p.n_boxes * kBoxN;
-#pragma unroll 1
-                for (int c = 0; c < ncols; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld_32cols(taddr + c, r);
-                    tmem_ld_wait();
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-                    }
-                }
-            }
+            if (kSwiGLU)
+                epilogue_swiglu(taddr, valid, reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                  grow * p.n_out + ti.n0);
+            else
+                epilogue_store_f32(taddr, valid, reinterpret_cast<float*>(p.out) +
+                                                     grow * p.n_out + ti.n0,
+                                   p.n_boxes * kBoxN);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -332,6 +344,250 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- CTA-pair kernel
+// Same roles and tile enumeration, but a cluster of two CTAs on two SMs works on
+// a 256-row tile with one tcgen05 MMA of M = 256 (cta_group::2): CTA rank r
+// holds A rows [128r, 128r+128) of the tile and half of the B columns (GEMM1:
+// rank 0 the W1 columns, rank 1 the W3 columns; GEMM2: column halves of W2),
+// and receives its own 128 rows of D in its TMEM.  Per CTA a stage is 32 KB
+// (A 16 KB + half of B 16 KB) instead of 48 KB, so six stages fit, and each
+// SM reads half as many B bytes per MMA.
+//
+// Synchronisation: both CTAs' TMA loads count their bytes on the leader's
+// (rank 0) full barrier, which only the leader arms with the bytes of both;
+// the leader's single MMA thread commits each consumed stage to the empty
+// barriers of both CTAs and each finished accumulator to the acc_full barriers
+// of both; the epilogue warps of both CTAs arrive on the leader's acc_empty
+// barrier (count 8).  Cluster barriers at start (barrier initialisation) and
+// end (before the pair frees its tensor memory) are reached by every thread of
+// both CTAs unconditionally; every mbarrier wait in between is bounded.
+constexpr int kPM = 256;                                       // rows per pair tile
+constexpr int kPairStages = 6;
+constexpr int kPairBBoxes = 2;                                 // B boxes per CTA per stage (max)
+constexpr int kPairStageBytes = kABytes + kPairBBoxes * kBBoxBytes;   // 32 KB
+constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + 1024;
+constexpr int kPairMinRows = 512;
+
+template <bool kSwiGLU>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB0,
+                            const __grid_constant__ CUtensorMap tmB1, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    __shared__ uint64_t full_bar[kPairStages];
+    __shared__ uint64_t empty_bar[kPairStages];
+    __shared__ uint64_t acc_full[2];
+    __shared__ uint64_t acc_empty[2];
+    __shared__ uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int s_off[kMaxE + 1];
+    __shared__ int s_mt[kMaxE + 1];
+    __shared__ volatile int s_abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 8);
+        }
+        mbar_init(&drain_bar, 1);
+        fence_barrier_init();
+        s_abort = 0;
+        int acc = 0;
+        s_mt[0] = 0;
+        for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+        for (int e = 0; e < p.E; ++e) {
+            const int cnt = max(0, s_off[e + 1] - s_off[e]);
+            acc += (cnt + kPM - 1) / kPM;
+            s_mt[e + 1] = acc;
+        }
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB0);
+        if (kSwiGLU) tma_prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync_all();  // the peer's barriers are initialised before anyone signals them
+    tc_fence_after_sync();
+    const uint32_t tmem_base = tmem_slot;
+
+    const int n_tiles = p.n_out / p.n_tile_out;
+    const int total_tiles = s_mt[p.E] * n_tiles;
+    const int kb_count = p.K / kBK;
+    const int boxes = p.n_boxes;  // B boxes per CTA per stage
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer (both CTAs)
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_parity = 0;
+            int issued = 0;
+            bool ok = true;
+            const uint32_t tx_pair = 2u * (kABytes + boxes * kBBoxBytes);
+            const uint32_t leader_full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
+            for (int t = pair; t < total_tiles && ok; t += npairs) {
+                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM);
+                const int my_row0 = ti.row0 + (int)rank * kBM;
+                const int wrow0 = ti.e * p.K;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (p.stall_after >= 0 && issued >= p.stall_after) {
+                        ok = false;  // test hook: both producers stop at the same stage
+                        break;
+                    }
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns) || s_abort) {
+                        record_error(p.err, kDeviceTimeoutBase | kRoleProducer);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sA = smem + stage * kPairStageBytes;
+                    uint8_t* sB = sA + kABytes;
+                    const uint32_t bar = leader_full0 + stage * (uint32_t)sizeof(uint64_t);
+                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx_pair);
+                    tma_load_2d_pair(sA, &tmA, bar, kb * kBK, my_row0);
+                    const int wrow = wrow0 + kb * kBK;
+                    if (kSwiGLU) {
+                        const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
+                        tma_load_2d_pair(sB, mb, bar, ti.n0, wrow);
+                        tma_load_2d_pair(sB + kBBoxBytes, mb, bar, ti.n0 + kBoxN, wrow);
+                    } else {
+                        const int c0 = ti.n0 + (int)rank * boxes * kBoxN;
+                        for (int j = 0; j < boxes; ++j)
+                            tma_load_2d_pair(sB + j * kBBoxBytes, &tmB0, bar, c0 + j * kBoxN, wrow);
+                    }
+                    issued_mask |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    ++issued;
+                    if (++stage == kPairStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) s_abort = 1;
+            // The leader's full barriers count the bytes of both CTAs: once every
+            // phase the leader armed has completed, no copy of either CTA is in flight.
+            if (leader)
+                for (int s = 0; s < kPairStages; ++s)
+                    if (issued_mask & (1u << s))
+                        (void)mbar_wait(&full_bar[s], (issued_parity >> s) & 1u, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (leader only)
+            const uint32_t idesc = idesc_bf16_f32(kPM, 2 * boxes * kBoxN, false, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < total_tiles && ok; t += npairs) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns) || s_abort) {
+                    record_error(p.err, kDeviceTimeoutBase | kRoleMma);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kAccCols;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, p.timeout_ns) || s_abort) {
+                        record_error(p.err, kDeviceTimeoutBase | kRoleMma);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * kPairStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t adesc = desc_kmajor_sw128(a_addr + kk * 32);
+                        const uint64_t bdesc = desc_mnmajor_sw128(b_addr + kk * 2048, kBBoxBytes);
+                        tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0);
+                    }
+                    const uint32_t e_own = smem_u32(&empty_bar[stage]);
+                    tc_commit_pair(e_own);
+                    tc_commit_pair(map_to_cta(e_own, 1));
+                    if (++stage == kPairStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                const uint32_t f_own = smem_u32(&acc_full[acc]);
+                tc_commit_pair(f_own);
+                tc_commit_pair(map_to_cta(f_own, 1));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) s_abort = 1;
+            tc_commit_pair(smem_u32(&drain_bar));
+            (void)mbar_wait(&drain_bar, 0, p.timeout_ns);
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        const int row_in_cta = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        const uint32_t leader_acc_empty0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
+        for (int t = pair; t < total_tiles; t += npairs) {
+            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM);
+            const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
+            if (!got || s_abort) {
+                if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
+                s_abort = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t taddr = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
+            const int row_in_tile = (int)rank * kBM + row_in_cta;
+            const bool valid = row_in_tile < ti.rows;
+            const int64_t grow = (int64_t)ti.row0 + row_in_tile;
+            if (kSwiGLU)
+                epilogue_swiglu(taddr, valid, reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                  grow * p.n_out + ti.n0);
+            else
+                epilogue_store_f32(taddr, valid, reinterpret_cast<float*>(p.out) +
+                                                     grow * p.n_out + ti.n0,
+                                   2 * boxes * kBoxN);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * (uint32_t)sizeof(uint64_t));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncwarp();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs are done with the pair's MMAs and tensor memory
+    tc_fence_after_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -389,6 +645,55 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Number of CTA pairs that can be resident at once (clusters must fit inside a
+// GPC, so this can be below half the SM count); cached per device.
+template <bool kSwiGLU>
+static int max_pairs() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev] == 0) {
+        auto kern = expert_gemm_pair_kernel<kSwiGLU>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kPairSmemBytes) != cudaSuccess)
+            return 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kPairSmemBytes;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        int n = 0;
+        // The kernel carries its cluster shape (2,1,1); ask without and, should the
+        // runtime want it spelled out, with the matching launch attribute.
+        if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess || n <= 0) {
+            (void)cudaGetLastError();
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess || n <= 0) {
+                (void)cudaGetLastError();
+                return 0;
+            }
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+template <bool kSwiGLU>
+static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const Params& p, int max_tiles, cudaStream_t stream) {
+    const int pairs = max_pairs<kSwiGLU>();  // also sets the shared-memory attribute
+    if (pairs <= 0) return MOE_ERR_CUDA;
+    const int grid = 2 * max(1, min(pairs, max_tiles));
+    expert_gemm_pair_kernel<kSwiGLU><<<grid, kThreads, kPairSmemBytes, stream>>>(a, b0, b1, p);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace gemm
 
 int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offsets, const void* W1,
@@ -405,8 +710,14 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
         !make_map(&m3, W3, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
         !make_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, kBK))
         return MOE_ERR_CUDA;
-    // Upper bound on m-tiles: sum over experts of ceil(rows_e / 128).
-    const int max_mtiles = (R + kBM - 1) / kBM + s.E;
+    // GEMM2 (long K = d_ff) runs on CTA pairs (256-row tiles, M = 256 MMAs) once
+    // there are at least kPairMinRows routed rows; GEMM1 (K = d, SwiGLU epilogue)
+    // stays on single CTAs with 128-row tiles, whose smaller padding of ragged
+    // expert groups outweighs the pair's saving (measured on the Mixtral shapes),
+    // and so does decode-sized work for both.
+    const bool pairs1 = false;
+    const bool pairs2 = R >= kPairMinRows;
+    auto mtiles = [&](int tile_rows) { return (R + tile_rows - 1) / tile_rows + s.E; };
 
     Params p1{};
     p1.offsets = offsets;
@@ -417,9 +728,11 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.K = s.d;
     p1.n_out = s.d_ff;
     p1.n_tile_out = 128;
-    p1.n_boxes = 4;
+    p1.n_boxes = pairs1 ? 2 : 4;  // per CTA: W1|W3 halves of a pair, or both on one CTA
     p1.stall_after = stall_after;
-    int rc = launch<true>(mx, m1, m3, p1, max_mtiles * (s.d_ff / 128), stream);
+    const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / 128);
+    int rc = pairs1 ? launch_pair<true>(mx, m1, m3, p1, t1, stream)
+                    : launch<true>(mx, m1, m3, p1, t1, stream);
     if (rc != MOE_OK) return rc;
     if (mid_event && cudaEventRecord(static_cast<cudaEvent_t>(mid_event), stream) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -429,9 +742,11 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.K = s.d_ff;
     p2.n_out = s.d;
     p2.n_tile_out = (s.d % 256 == 0) ? 256 : 128;
-    p2.n_boxes = p2.n_tile_out / kBoxN;
-    p2.stall_after = -1;
-    return launch<false>(mh, m2, m2, p2, max_mtiles * (s.d / p2.n_tile_out), stream);
+    p2.n_boxes = p2.n_tile_out / kBoxN / (pairs2 ? 2 : 1);
+    p2.stall_after = stall_after;
+    const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
+    return pairs2 ? launch_pair<false>(mh, m2, m2, p2, t2, stream)
+                  : launch<false>(mh, m2, m2, p2, t2, stream);
 }
 
 }  // namespace moe

@@ -215,8 +215,9 @@ def test_forward_deterministic_and_hostio_matches():
     assert torch.equal(y1.cpu(), y_host)
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
-    inp = workload_inputs("tiny")
+@pytest.mark.parametrize("T", [64, 300], ids=["single-cta", "cta-pair"])
+def test_bounded_wait_reports_timeout_and_context_survives(T):
+    inp = make_inputs(T, 128, 256, 8, 2, seed=44)
     T, d, d_ff, E, k = inp["shape"]
     o_idx, _, _ = oracle.route(inp["x"], inp["Wg"], E, k)
     r_off, r_perm, _ = oracle.dispatch(o_idx, E)
