@@ -12,7 +12,7 @@
 //     each expert, then each thread walks its run again and hands out positions
 //     in token order.  Integer-only and deterministic (no atomics on positions).
 //  2. scatter kernel: reads each x row once and writes it to its k sorted rows
-//     (16-byte vector copies, one warp per row).
+//     (16-byte vector copies, one thread per 16-byte chunk).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -92,39 +92,23 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
         }
 }
 
-// x_sorted[inv[t, s]] = x[t] for every slot s of token t.
+// x_sorted[inv[t, s]] = x[t] for every slot s of token t; one thread per
+// (token, 16-byte chunk), so x is read once and the k copies are written with
+// coalesced 16-byte stores however few tokens there are.
 __global__ void __launch_bounds__(256)
     scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv, int T, int chunks,
                    int k, uint4* __restrict__ x_sorted) {
-    const int lane = threadIdx.x & 31;
-    const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
-        int dst[8];
+    const int64_t total = (int64_t)T * chunks;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int t = (int)(i / chunks);
+        const int c = (int)(i - (int64_t)t * chunks);
+        const uint4 v = __ldg(x + i);
 #pragma unroll
-        for (int s = 0; s < 8; ++s) dst[s] = s < k ? inv[(int64_t)t * k + s] : -1;
-        const uint4* src = x + (int64_t)t * chunks;
-        int c = lane;
-        for (; c + 96 < chunks; c += 128) {
-            const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32);
-            const uint4 v2 = __ldg(src + c + 64), v3 = __ldg(src + c + 96);
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                if (s >= k) break;
-                if (dst[s] < 0) continue;
-                uint4* o = x_sorted + (int64_t)dst[s] * chunks + c;
-                o[0] = v0;
-                o[32] = v1;
-                o[64] = v2;
-                o[96] = v3;
-            }
-        }
-        for (; c < chunks; c += 32) {
-            const uint4 v = __ldg(src + c);
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                if (s >= k) break;
-                if (dst[s] >= 0) x_sorted[(int64_t)dst[s] * chunks + c] = v;
-            }
+        for (int s = 0; s < 8; ++s) {
+            if (s >= k) break;
+            const int dst = __ldg(inv + (int64_t)t * k + s);
+            if (dst >= 0) x_sorted[(int64_t)dst * chunks + c] = v;
         }
     }
 }
@@ -148,9 +132,9 @@ int launch_dispatch_scatter(const moe_shape& s, const void* x, const int32_t* in
                             cudaStream_t stream) {
     using namespace dispatch;
     if (s.T == 0) return MOE_OK;
-    const int warps_per_block = 256 / 32;
-    const int grid = std::max(1, std::min((s.T + warps_per_block - 1) / warps_per_block,
-                                          device_sm_count() * 8));
+    const int64_t work = (int64_t)s.T * (s.d / 8);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256,
+                                                                 (int64_t)device_sm_count() * 8));
     scatter_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(x), inv, s.T, s.d / 8, s.k,
                                              static_cast<uint4*>(x_sorted));
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

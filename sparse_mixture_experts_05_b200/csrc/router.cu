@@ -6,8 +6,10 @@
 //
 // The contraction x[T,d] . Wg[d,E] is skinny (E = 8) and HBM-bound on reading
 // x once; it runs on mma.sync m16n8k16 (bf16 in, fp32 accumulate) so the issue
-// slots stay free for loads.  A warp owns 16 tokens and a quarter of d; the four
-// quarter sums are added in a fixed order, so results are deterministic.
+// slots stay free for loads.  A warp owns 16 tokens and 1/KSPLIT of d; the
+// KSPLIT partial sums are added in a fixed order, so results are deterministic.
+// KSPLIT grows when there are few tokens (decode) so that more warps share the
+// one tile of 16 tokens and the kernel is not bound by one warp's load latency.
 //
 // k-permutation: a dot product may pair its terms in any order, so a lane loads
 // 8 consecutive x elements (one 16-byte load) and feeds them to two MMAs as
@@ -31,8 +33,6 @@ namespace moe {
 namespace router {
 
 constexpr int kWarps = 16;
-constexpr int kKSplit = 4;
-constexpr int kSlots = kWarps / kKSplit;  // token tiles of 16 per block iteration
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxK = 8;
 
@@ -50,14 +50,15 @@ __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
     return v > bv || (v == bv && id < bid) || bid == INT_MAX;
 }
 
-template <int NT>
+template <int NT, int KSPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
                   const float* __restrict__ bias, int T, int d, int E, int k,
                   int32_t* __restrict__ idx, float* __restrict__ gate,
                   float* __restrict__ logits) {
+    constexpr int kSlots = kWarps / KSPLIT;  // token tiles of 16 per block iteration
     extern __shared__ uint4 s_wg[];  // [d/32][NT][32 lanes] x 8 bf16
-    __shared__ float s_red[kSlots][kKSplit][NT][32][4];
+    __shared__ float s_red[kSlots][KSPLIT][NT][32][4];
 
     // Stage W_r in fragment order: entry (kb, nt, lane) holds
     // Wg[kb*32 + (lane&3)*8 + j][nt*8 + (lane>>2)] for j = 0..7 (zero for n >= E).
@@ -81,11 +82,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int slot = warp / kKSplit;
-    const int kq = warp % kKSplit;
+    const int slot = warp / KSPLIT;
+    const int kq = warp % KSPLIT;
     const int g = lane >> 2;
     const int t4 = lane & 3;
-    const int kper = d / kKSplit;
+    const int kper = d / KSPLIT;
     const int ntiles = (T + 15) / 16;
 
     for (int base = blockIdx.x * kSlots; base < ntiles; base += gridDim.x * kSlots) {
@@ -126,9 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     float sum = s_red[slot][0][nt][lane][i];
-                    sum = __fadd_rn(sum, s_red[slot][1][nt][lane][i]);
-                    sum = __fadd_rn(sum, s_red[slot][2][nt][lane][i]);
-                    sum = __fadd_rn(sum, s_red[slot][3][nt][lane][i]);
+#pragma unroll
+                    for (int q = 1; q < KSPLIT; ++q) sum = __fadd_rn(sum, s_red[slot][q][nt][lane][i]);
                     const int n = nt * 8 + 2 * t4 + (i & 1);
                     if (bias && n < E) sum = __fadd_rn(sum, bias[n]);
                     v[nt][i] = sum;
@@ -213,19 +213,33 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
     const int NT = (s.E + 7) / 8;
     const size_t smem = (size_t)s.d * NT * 16;
     const int ntiles = (s.T + 15) / 16;
-    const int grid = std::max(1, std::min(device_sm_count(), (ntiles + kSlots - 1) / kSlots));
+    const int sms = device_sm_count();
+    // Largest split of d (into 16, 8 or 4 parts, each a whole number of 32-wide
+    // k blocks) that still needs no more CTAs than there are SMs: few tokens
+    // (decode) then get 16 warps per tile instead of 4.
+    int ksplit = 4;
+    for (int cand : {16, 8}) {
+        const int ctas = (ntiles * cand + kWarps - 1) / kWarps;
+        if ((s.d / 32) % cand == 0 && ctas <= sms) {
+            ksplit = cand;
+            break;
+        }
+    }
+    const int slots = kWarps / ksplit;
+    const int grid = std::max(1, std::min(sms, (ntiles + slots - 1) / slots));
     const uint16_t* xp = static_cast<const uint16_t*>(x);
     const uint16_t* wp = static_cast<const uint16_t*>(Wg);
-#define MOE_ROUTER_CASE(N)                                                                      \
-    case N: {                                                                                   \
-        auto kern = router_kernel<N>;                                                           \
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
-                                 (int)smem) != cudaSuccess)                                     \
-            return MOE_ERR_CUDA;                                                                \
-        kern<<<grid, kThreads, smem, stream>>>(xp, wp, bias, s.T, s.d, s.E, s.k, idx, gate,     \
-                                               logits);                                        \
-        break;                                                                                  \
-    }
+    auto run = [&](auto kern) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        kern<<<grid, kThreads, smem, stream>>>(xp, wp, bias, s.T, s.d, s.E, s.k, idx, gate, logits);
+        return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    };
+#define MOE_ROUTER_CASE(N)                                                  \
+    case N:                                                                 \
+        return ksplit == 16 ? run(router_kernel<N, 16>)                     \
+               : ksplit == 8 ? run(router_kernel<N, 8>) : run(router_kernel<N, 4>);
     switch (NT) {
         MOE_ROUTER_CASE(1)
         MOE_ROUTER_CASE(2)
@@ -235,7 +249,6 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
             return MOE_ERR_UNSUPPORTED;
     }
 #undef MOE_ROUTER_CASE
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe
