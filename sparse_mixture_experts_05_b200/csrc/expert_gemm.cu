@@ -95,14 +95,16 @@ __device__ __forceinline__ TileInfo decode_tile_rows(int t, const int* mt_prefix
     return ti;
 }
 
-// GEMM1 epilogue of one TMEM lane (= one row): columns [0,128) hold a = x W1,
-// columns [128,256) hold b = x W3; h = SiLU(a) * b = a / (1 + exp(-a)) * b.
-__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, __nv_bfloat16* hrow) {
+// GEMM1 epilogue of one TMEM lane (= one row): columns [0, hcols) hold
+// a = x W1, columns [hcols, 2 hcols) hold b = x W3 for the same output columns;
+// h = SiLU(a) * b = a / (1 + exp(-a)) * b.
+__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, __nv_bfloat16* hrow,
+                                                int hcols) {
 #pragma unroll 1
-    for (int c = 0; c < kAccCols / 2; c += 32) {
+    for (int c = 0; c < hcols; c += 32) {
         uint32_t ra[32], rb[32];
         tmem_ld_32cols(taddr + c, ra);
-        tmem_ld_32cols(taddr + kAccCols / 2 + c, rb);
+        tmem_ld_32cols(taddr + hcols + c, rb);
         tmem_ld_wait();
         if (valid) {
             uint32_t packed[16];
@@ -232,11 +234,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(sA, &tmA, &full_bar[stage], kb * kBK, ti.row0);
                     const int wrow = wrow0 + kb * kBK;
                     if (kSwiGLU) {
-                        tma_load_2d(sB, &tmB0, &full_bar[stage], ti.n0, wrow);
-                        tma_load_2d(sB + kBBoxBytes, &tmB0, &full_bar[stage], ti.n0 + kBoxN, wrow);
-                        tma_load_2d(sB + 2 * kBBoxBytes, &tmB1, &full_bar[stage], ti.n0, wrow);
-                        tma_load_2d(sB + 3 * kBBoxBytes, &tmB1, &full_bar[stage], ti.n0 + kBoxN,
-                                    wrow);
+                        // W1 columns [n0, n0 + half) then the same W3 columns
+                        const int half = p.n_boxes / 2;
+                        for (int j = 0; j < half; ++j) {
+                            tma_load_2d(sB + j * kBBoxBytes, &tmB0, &full_bar[stage],
+                                        ti.n0 + j * kBoxN, wrow);
+                            tma_load_2d(sB + (half + j) * kBBoxBytes, &tmB1, &full_bar[stage],
+                                        ti.n0 + j * kBoxN, wrow);
+                        }
                     } else {
                         for (int j = 0; j < p.n_boxes; ++j)
                             tma_load_2d(sB + j * kBBoxBytes, &tmB0, &full_bar[stage],
@@ -325,7 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
             if (kSwiGLU)
                 epilogue_swiglu(taddr, valid, reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                                  grow * p.n_out + ti.n0);
+                                                  grow * p.n_out + ti.n0,
+                                p.n_tile_out);
             else
                 epilogue_store_f32(taddr, valid, reinterpret_cast<float*>(p.out) +
                                                      grow * p.n_out + ti.n0,
@@ -567,7 +573,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
             if (kSwiGLU)
                 epilogue_swiglu(taddr, valid, reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                                  grow * p.n_out + ti.n0);
+                                                  grow * p.n_out + ti.n0,
+                                p.n_tile_out);
             else
                 epilogue_store_f32(taddr, valid, reinterpret_cast<float*>(p.out) +
                                                      grow * p.n_out + ti.n0,
@@ -727,10 +734,14 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.E = s.E;
     p1.K = s.d;
     p1.n_out = s.d_ff;
+    // GEMM1 tiles cover 128 h columns: 2 weight boxes of W1 and 2 of W3 on one
+    // CTA (or one matrix per CTA of a pair).  Narrower 64-column tiles, which
+    // balance small batches across the SMs better, were measured slower at
+    // decode: every tile also streams a full 128-row A tile.
     p1.n_tile_out = 128;
-    p1.n_boxes = pairs1 ? 2 : 4;  // per CTA: W1|W3 halves of a pair, or both on one CTA
+    p1.n_boxes = pairs1 ? 2 : 4;  // per CTA
     p1.stall_after = stall_after;
-    const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / 128);
+    const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / p1.n_tile_out);
     int rc = pairs1 ? launch_pair<true>(mx, m1, m3, p1, t1, stream)
                     : launch<true>(mx, m1, m3, p1, t1, stream);
     if (rc != MOE_OK) return rc;
