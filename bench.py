@@ -393,8 +393,10 @@ def run_ours(a):
     roof["kernel"] = ("expert_gemm_kernel (two launches per step: GEMM1 x.W1|x.W3 -> SiLU(a)*b, "
                       "GEMM2 h.W2); achieved = algorithmic units of both launches / their summed "
                       "CUDA-event time")
-    traffic = committed_traffic(a.workload)
+    traffic = committed_traffic(a.workload) if a.tokens is None and a.experts is None else None
     roof["traffic"] = traffic
+    roof["traffic_scope"] = ("DRAM bytes of both expert_gemm launches of one step, from the committed "
+                             "ncu capture of the same kernel source (null once the source changed)")
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
