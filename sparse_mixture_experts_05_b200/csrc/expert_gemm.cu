@@ -32,6 +32,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -70,6 +71,7 @@ struct Params {
     int n_tile_out;          // output columns per tile
     int n_boxes;             // B boxes per stage (MMA N = 64 * n_boxes)
     int stall_after;         // test hook: producer stops after this many stages (-1: never)
+    int group_m;             // m-tiles per rasterisation group (see decode_tile_rows)
 };
 
 struct TileInfo {
@@ -77,17 +79,26 @@ struct TileInfo {
 };
 
 // Tile t of the expert-major enumeration: expert e owns tiles
-// [n_tiles * mt_prefix[e], n_tiles * mt_prefix[e+1]), n-major within an
-// expert with m fastest, so tiles that run at the same time share weight tiles.
+// [n_tiles * mt_prefix[e], n_tiles * mt_prefix[e+1]).  Within an expert the
+// m-tiles are walked in groups of `group_m` (the last group may be smaller);
+// within a group the order is n-major with m fastest.  Tiles that run at the
+// same time then share weight tiles, and a group's activation rows -- sized on
+// the host to sit in L2 next to the weight stream -- are read from DRAM once
+// for all column tiles instead of once per few column tiles.
 __device__ __forceinline__ TileInfo decode_tile_rows(int t, const int* mt_prefix, const int* off,
-                                                     int n_tiles, int n_tile_out, int tile_rows) {
+                                                     int n_tiles, int n_tile_out, int tile_rows,
+                                                     int group_m) {
     TileInfo ti;
     int e = 0;
     while (t >= n_tiles * mt_prefix[e + 1]) ++e;
     const int local = t - n_tiles * mt_prefix[e];
     const int mt = mt_prefix[e + 1] - mt_prefix[e];
-    const int n = local / mt;
-    const int m = local - n * mt;
+    const int g = local / (group_m * n_tiles);
+    const int m0 = g * group_m;
+    const int gm = min(group_m, mt - m0);
+    const int r = local - g * group_m * n_tiles;
+    const int n = r / gm;
+    const int m = m0 + (r - n * gm);
     ti.e = e;
     ti.row0 = off[e] + m * tile_rows;
     ti.rows = min(tile_rows, off[e + 1] - ti.row0);
@@ -216,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             const uint32_t tx_bytes = kABytes + p.n_boxes * kBBoxBytes;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM);
+                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM, p.group_m);
                 const int wrow0 = ti.e * p.K;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (p.stall_after >= 0 && issued >= p.stall_after) {
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM);
+            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM, p.group_m);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
                 if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
@@ -455,7 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t tx_pair = 2u * (kABytes + boxes * kBBoxBytes);
             const uint32_t leader_full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
             for (int t = pair; t < total_tiles && ok; t += npairs) {
-                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM);
+                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM, p.group_m);
                 const int my_row0 = ti.row0 + (int)rank * kBM;
                 const int wrow0 = ti.e * p.K;
                 for (int kb = 0; kb < kb_count; ++kb) {
@@ -559,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         const uint32_t leader_acc_empty0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
         for (int t = pair; t < total_tiles; t += npairs) {
-            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM);
+            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM, p.group_m);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
                 if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
@@ -725,6 +736,12 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     const bool pairs1 = false;
     const bool pairs2 = R >= kPairMinRows;
     auto mtiles = [&](int tile_rows) { return (R + tile_rows - 1) / tile_rows + s.E; };
+    // m-tiles per rasterisation group: as many as keep the group's activation
+    // rows (tile_rows x K bf16 each) within ~48 MB of the 126 MB L2.
+    auto group_rows = [](int tile_rows, int K) {
+        const int64_t per_tile = (int64_t)tile_rows * K * 2;
+        return (int)std::max<int64_t>(1, (int64_t(48) << 20) / per_tile);
+    };
 
     Params p1{};
     p1.offsets = offsets;
@@ -741,6 +758,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.n_tile_out = 128;
     p1.n_boxes = pairs1 ? 2 : 4;  // per CTA
     p1.stall_after = stall_after;
+    p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
     const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / p1.n_tile_out);
     int rc = pairs1 ? launch_pair<true>(mx, m1, m3, p1, t1, stream)
                     : launch<true>(mx, m1, m3, p1, t1, stream);
@@ -755,6 +773,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.n_tile_out = (s.d % 256 == 0) ? 256 : 128;
     p2.n_boxes = p2.n_tile_out / kBoxN / (pairs2 ? 2 : 1);
     p2.stall_after = stall_after;
+    p2.group_m = group_rows(pairs2 ? kPM : kBM, s.d_ff);
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
     return pairs2 ? launch_pair<false>(mh, m2, m2, p2, t2, stream)
                   : launch<false>(mh, m2, m2, p2, t2, stream);
