@@ -67,6 +67,8 @@ def _load():
         lib.orc_forward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, P]
         lib.orc_forward_tokens.restype = I
         lib.orc_forward_tokens.argtypes = [I, P, I, I, I, I, I, P, P, P, P, P, P, I, P, P, P]
+        lib.orc_aux_loss.restype = ctypes.c_double
+        lib.orc_aux_loss.argtypes = [I, I, I, P, P, P, P, P]
         lib.orc_param_count.restype = None
         lib.orc_param_count.argtypes = [I64] * 9 + [I, P, P]
         _lib = lib
@@ -216,6 +218,19 @@ def forward_tokens(tokens, x, wg, W1, W3, W2, k: int, bias=None, round_h: bool =
     if rc:
         raise ValueError(f"orc_forward_tokens failed (rc={rc})")
     return y, idx, gate
+
+
+def aux_loss(logits, idx, mask=None):
+    """Load-balancing auxiliary term E * sum_s sum_i f_{s,i} P_i.  Returns (aux, f [k,E], P [E])."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, E = logits.shape
+    k = idx.shape[1]
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    f = np.empty((k, E), np.float64)
+    P = np.empty(E, np.float64)
+    aux = _load().orc_aux_loss(T, E, k, _p(logits), _p(idx), _p(m), _p(f), _p(P))
+    return aux, f, P
 
 
 def param_count(V, d, L, H, G, dh, d_ff, E, k, bias=False):

@@ -344,3 +344,51 @@ void orc_param_count(int64_t V, int64_t d, int64_t L, int64_t H, int64_t G, int6
     *total = embed + L * (attn + router + E * expert + norms) + d + head;
     *active = embed + L * (attn + router + k * expert + norms) + d + head;
 }
+
+/* ---- load-balancing auxiliary loss -------------------------------------------
+ * Mixtral page, section "Load-balancing loss":
+ *     aux = E * sum_{s<k} sum_{i<E} f_{s,i} * P_i
+ * f_{s,i}: fraction of the counted tokens whose top-k slot s holds expert i;
+ * P_i:     mean over the counted tokens of the softmax over all E router
+ *          logits, entry i.
+ * (the training loss adds alpha * aux; under uniform load aux = k.)
+ * Counted tokens are all T, or those with mask[t] != 0 when mask is given
+ * (padding excluded).  f [k*E] and P [E] are written when non-null.  Returns
+ * aux (0 when no token is counted). */
+double orc_aux_loss(int T, int E, int k, const float* logits, const int32_t* idx,
+                    const uint8_t* mask, double* f_out, double* P_out) {
+    double* f = (double*)calloc((size_t)k * E, sizeof(double));
+    double* P = (double*)calloc((size_t)E, sizeof(double));
+    double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    double n = 0.0;
+    for (int t = 0; t < T; ++t) {
+        if (mask && !mask[t]) continue;
+        n += 1.0;
+        const float* g = logits + (int64_t)t * E;
+        double m = (double)g[0];
+        for (int e = 1; e < E; ++e)
+            if ((double)g[e] > m) m = (double)g[e];
+        double den = 0.0;
+        for (int e = 0; e < E; ++e) {
+            p[e] = exp((double)g[e] - m);
+            den += p[e];
+        }
+        for (int e = 0; e < E; ++e) P[e] += p[e] / den;
+        for (int s = 0; s < k; ++s) {
+            const int e = idx[(int64_t)t * k + s];
+            if (e >= 0 && e < E) f[(int64_t)s * E + e] += 1.0;
+        }
+    }
+    double aux = 0.0;
+    if (n > 0) {
+        for (int i = 0; i < k * E; ++i) f[i] /= n;
+        for (int e = 0; e < E; ++e) P[e] /= n;
+        for (int s = 0; s < k; ++s)
+            for (int e = 0; e < E; ++e) aux += f[(int64_t)s * E + e] * P[e];
+        aux *= (double)E;
+    }
+    if (f_out) memcpy(f_out, f, sizeof(double) * (size_t)k * E);
+    if (P_out) memcpy(P_out, P, sizeof(double) * (size_t)E);
+    free(f); free(P); free(p);
+    return aux;
+}

@@ -344,3 +344,48 @@ def test_planted_mistakes_fail_the_pins():
     W2t = sq["W2"].transpose(1, 2).contiguous()
     y_t, _, _ = oracle.forward(sq["x"], sq["Wg"], sq["W1"], sq["W3"], W2t, 1, round_h=False)
     assert np.max(np.abs(y_t - ref_sq)) > 1e-3 * np.max(np.abs(ref_sq))
+
+
+# ---------------------------------------------------------------- load-balancing loss
+def test_aux_loss_is_k_under_uniform_load():
+    """Section "Load-balancing loss": under uniform load the auxiliary term equals k."""
+    E, T = 8, 64
+    for k in (1, 2, 3):
+        logits = np.zeros((T, E), np.float32)                 # P_i = 1/E
+        idx = np.array([[(t + s) % E for s in range(k)] for t in range(T)], np.int32)  # f = 1/E
+        aux, f, P = oracle.aux_loss(logits, idx)
+        assert aux == pytest.approx(k, abs=1e-12)
+        assert np.allclose(f, 1 / E) and np.allclose(P, 1 / E)
+
+
+def test_aux_loss_closed_form_for_collapsed_routing_and_masking():
+    E, T = 8, 40
+    logits = np.full((T, E), -1e30, np.float32)
+    logits[:, :2] = 0.0                                      # P = (1/2, 1/2, 0, ...)
+    idx = np.tile(np.array([[0, 1]], np.int32), (T, 1))      # f_{0,0} = f_{1,1} = 1
+    aux, _, P = oracle.aux_loss(logits, idx)
+    assert aux == pytest.approx(E, abs=1e-12)                # E * (1 * 1/2 + 1 * 1/2)
+    # padding tokens are not counted: append garbage rows with mask 0
+    rng = np.random.default_rng(0)
+    lg2 = np.concatenate([logits, rng.standard_normal((10, E)).astype(np.float32)])
+    id2 = np.concatenate([idx, rng.integers(0, E, (10, 2)).astype(np.int32)])
+    mask = np.concatenate([np.ones(T, np.uint8), np.zeros(10, np.uint8)])
+    aux2, _, _ = oracle.aux_loss(lg2, id2, mask)
+    assert aux2 == pytest.approx(E, abs=1e-12)
+
+
+def test_aux_loss_matches_brute_force_definition():
+    rng = np.random.default_rng(1)
+    T, E, k = 37, 8, 2
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    idx, _, _ = oracle.route(make_inputs(T, 64, 128, E, k, seed=2)["x"],
+                             make_inputs(T, 64, 128, E, k, seed=2)["Wg"], E, k)
+    aux, f, P = oracle.aux_loss(logits, idx)
+    # explicit double sums over (token, slot, expert) with scipy's softmax
+    from scipy.special import softmax
+    p = softmax(logits.astype(np.float64), axis=1)
+    want = 0.0
+    for s in range(k):
+        for i in range(E):
+            want += np.mean(idx[:, s] == i) * np.mean(p[:, i])
+    assert aux == pytest.approx(E * want, rel=1e-12)
