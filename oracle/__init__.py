@@ -67,6 +67,11 @@ def _load():
         lib.orc_forward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, P]
         lib.orc_forward_tokens.restype = I
         lib.orc_forward_tokens.argtypes = [I, P, I, I, I, I, I, P, P, P, P, P, P, I, P, P, P]
+        lib.orc_rmsnorm.restype = None
+        lib.orc_rmsnorm.argtypes = [I, I, P, P, ctypes.c_double, P]
+        lib.orc_block_forward.restype = I
+        lib.orc_block_forward.argtypes = [I, I, I, I, I, P, P, ctypes.c_double, P, P, P, P, P, I,
+                                          P, P, P]
         lib.orc_aux_loss.restype = ctypes.c_double
         lib.orc_aux_loss.argtypes = [I, I, I, P, P, P, P, P]
         lib.orc_param_count.restype = None
@@ -218,6 +223,38 @@ def forward_tokens(tokens, x, wg, W1, W3, W2, k: int, bias=None, round_h: bool =
     if rc:
         raise ValueError(f"orc_forward_tokens failed (rc={rc})")
     return y, idx, gate
+
+
+def rmsnorm(U, gamma, eps: float = 1e-5):
+    """bf16(U / sqrt(mean(U^2) + eps) * gamma) row by row; returns uint16 bit patterns."""
+    U = _u16(U)
+    gamma = _u16(gamma)
+    T, d = U.shape
+    u = np.empty((T, d), np.uint16)
+    _load().orc_rmsnorm(T, d, _p(U), _p(gamma), float(eps), _p(u))
+    return u
+
+
+def block_forward(U, gamma, wg, W1, W3, W2, k: int, eps: float = 1e-5, bias=None,
+                  round_h: bool = True):
+    """H = U + MoE(RMSNorm(U)) (float64, unrounded).  Returns (H, idx, gate)."""
+    U = _u16(U)
+    gamma = _u16(gamma)
+    wg = _u16(wg)
+    W1 = _u16(W1)
+    W3 = _u16(W3)
+    W2 = _u16(W2)
+    T, d = U.shape
+    E, _, d_ff = W1.shape
+    H = np.empty((T, d), np.float64)
+    idx = np.empty((T, k), np.int32)
+    gate = np.empty((T, k), np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    rc = _load().orc_block_forward(T, d, d_ff, E, k, _p(U), _p(gamma), float(eps), _p(wg), _p(b),
+                                   _p(W1), _p(W3), _p(W2), int(round_h), _p(H), _p(idx), _p(gate))
+    if rc:
+        raise ValueError(f"orc_block_forward failed (rc={rc})")
+    return H, idx, gate
 
 
 def aux_loss(logits, idx, mask=None):

@@ -392,3 +392,40 @@ double orc_aux_loss(int T, int E, int k, const float* logits, const int32_t* idx
     free(f); free(P); free(p);
     return aux;
 }
+
+/* ---- block edges: RMSNorm before the layer, residual after it ------------------
+ * Mixtral page, section "Прямой проход в формулах":
+ *     H = U + MoE(RMSNorm_2(U)),   RMSNorm(z) = z / sqrt(mean_j z_j^2 + eps) (.) gamma
+ * (eps = rms_norm_eps, 1e-5 for Mixtral 8x7B).  The normalised rows are the
+ * bf16 input of the layer, so they are rounded to bf16 (nearest even).
+ *   U [T,d] bf16, gamma [d] bf16 -> u [T,d] bf16 bits. */
+void orc_rmsnorm(int T, int d, const uint16_t* U, const uint16_t* gamma, double eps, uint16_t* u) {
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const uint16_t* z = U + (int64_t)t * d;
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j) {
+            const double v = orc_bf16_value(z[j]);
+            ss += v * v;
+        }
+        const double r = sqrt(ss / d + eps);
+        for (int j = 0; j < d; ++j)
+            u[(int64_t)t * d + j] = orc_bf16_bits(orc_bf16_value(z[j]) / r * orc_bf16_value(gamma[j]));
+    }
+}
+
+/* H = U + MoE(RMSNorm(U)) with the layer of orc_forward (H unrounded, double). */
+int orc_block_forward(int T, int d, int d_ff, int E, int k, const uint16_t* U, const uint16_t* gamma,
+                      double eps, const uint16_t* wg, const float* bias, const uint16_t* W1,
+                      const uint16_t* W3, const uint16_t* W2, int round_h, double* H,
+                      int32_t* idx_out, float* gate_out) {
+    uint16_t* u = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(T > 0 ? T : 1) * d);
+    if (!u) return 2;
+    orc_rmsnorm(T, d, U, gamma, eps, u);
+    const int rc = orc_forward(T, d, d_ff, E, k, u, wg, bias, W1, W3, W2, round_h, H, idx_out,
+                               gate_out);
+    if (!rc)
+        for (int64_t i = 0; i < (int64_t)T * d; ++i) H[i] += orc_bf16_value(U[i]);
+    free(u);
+    return rc;
+}

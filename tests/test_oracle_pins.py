@@ -389,3 +389,55 @@ def test_aux_loss_matches_brute_force_definition():
         for i in range(E):
             want += np.mean(idx[:, s] == i) * np.mean(p[:, i])
     assert aux == pytest.approx(E * want, rel=1e-12)
+
+
+# ---------------------------------------------------------------- block edges (RMSNorm, residual)
+def _bf16(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def test_rmsnorm_closed_forms():
+    d = 256
+    # constant row c, gamma = 1: c / sqrt(c^2 + eps)
+    for c in (0.5, -3.0, 1e-3):
+        U = _bf16(np.full((1, d), c))
+        u = oracle.bf16_to_f64(oracle.rmsnorm(U, _bf16(np.ones(d)), eps=1e-5))
+        cv = float(_bf16([c])[0])
+        want = oracle.bf16_to_f64(oracle.round_bf16(np.array([cv / math.sqrt(cv * cv + 1e-5)])))[0]
+        assert np.all(u == want)
+    # with eps = 0 the output is scale-free and has unit mean square before rounding
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((4, d))
+    u1 = oracle.bf16_to_f64(oracle.rmsnorm(_bf16(z), _bf16(np.ones(d)), eps=0.0))
+    u2 = oracle.bf16_to_f64(oracle.rmsnorm(_bf16(4 * z), _bf16(np.ones(d)), eps=0.0))  # 4x: exact in bf16
+    assert np.array_equal(u1, u2)
+    assert np.allclose(np.mean(u1 ** 2, axis=1), 1.0, atol=1e-2)
+    # gamma scales column j; gamma = 0 gives zeros
+    g = np.linspace(-2, 2, d)
+    ug = oracle.bf16_to_f64(oracle.rmsnorm(_bf16(z), _bf16(g), eps=0.0))
+    assert np.max(np.abs(ug - u1 * oracle.bf16_to_f64(oracle.round_bf16(g)))) <= 0.02 * np.max(np.abs(ug))
+    assert np.all(oracle.bf16_to_f64(oracle.rmsnorm(_bf16(z), _bf16(np.zeros(d)))) == 0)
+
+
+def test_block_residual_passes_through_when_the_layer_is_zero():
+    inp = make_inputs(30, 128, 256, 8, 2, seed=50)
+    gamma = _bf16(np.ones(128))
+    zero_W2 = torch.zeros_like(inp["W2"])
+    H, _, _ = oracle.block_forward(inp["x"], gamma, inp["Wg"], inp["W1"], inp["W3"], zero_W2, 2)
+    assert np.array_equal(H, _f64(inp["x"]))
+    H0, idx0, _ = oracle.block_forward(inp["x"], _bf16(np.zeros(128)), inp["Wg"], inp["W1"],
+                                       inp["W3"], inp["W2"], 2)
+    assert np.array_equal(H0, _f64(inp["x"]))          # u = 0 -> h = SiLU(0) * 0 = 0
+    assert np.all(idx0 == np.array([0, 1]))            # all logits 0: ties go to the lower index
+
+
+def test_block_equals_residual_plus_layer_of_the_normalised_rows():
+    inp = make_inputs(40, 128, 256, 8, 2, seed=51, bias=True)
+    rng = np.random.default_rng(4)
+    gamma = _bf16(1 + 0.1 * rng.standard_normal(128))
+    u = oracle.rmsnorm(inp["x"], gamma)
+    y, idx, _ = oracle.forward(u, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], 2, bias=inp["bias"])
+    H, idx2, _ = oracle.block_forward(inp["x"], gamma, inp["Wg"], inp["W1"], inp["W3"], inp["W2"],
+                                      2, bias=inp["bias"])
+    assert np.array_equal(idx, idx2)
+    assert np.array_equal(H, _f64(inp["x"]) + y)
