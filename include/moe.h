@@ -172,6 +172,22 @@ int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float
                          size_t ws_bytes, void* const* events, int n_events, void* stream);
 
 /*
+ * moe_block_forward -- the MoE half of a decoder block with its edges
+ * (Mixtral textbook page, section "Прямой проход в формулах"):
+ *     H = U + MoE(RMSNorm_2(U)),   RMSNorm(z) = z / sqrt(mean_j z_j^2 + eps) (.) gamma
+ *   U [T,d] bf16: the residual stream after attention (in)
+ *   gamma [d] bf16: RMSNorm_2 scale; eps >= 0 (rms_norm_eps, 1e-5 for Mixtral) (in)
+ *   Wg, bias, W1, W3, W2 as for moe_forward (in);  H [T,d] bf16 (out)
+ *   ws: >= moe_block_workspace_bytes(s) bytes of device memory
+ * The normalised rows are rounded to bf16 (the layer's input); the residual is
+ * added in float32 to the combined expert outputs before the one rounding of H.
+ */
+size_t moe_block_workspace_bytes(moe_shape s);
+int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, const void* Wg,
+                      const float* bias, const void* W1, const void* W3, const void* W2, void* H,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_forward_hostio -- moe_forward with x and y in HOST memory (pinned memory
  * gives asynchronous copies): enqueues the host->device copy of x into the
  * workspace, the layer, and the device->host copy of y, all on `stream`.  The
@@ -183,6 +199,24 @@ size_t moe_forward_hostio_workspace_bytes(moe_shape s);
 int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const float* bias,
                        const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
                        size_t ws_bytes, void* stream);
+
+/*
+ * moe_aux_loss -- load-balancing auxiliary term of the router (Mixtral textbook
+ * page, section "Load-balancing loss"):
+ *     aux = E * sum_{s<k} sum_{i<E} f_{s,i} * P_i
+ * f_{s,i}: fraction of the counted tokens whose top-k slot s holds expert i;
+ * P_i: mean over the counted tokens of the softmax over all E router logits.
+ * The training loss adds alpha * aux (alpha = router_aux_loss_coef); under
+ * uniform load aux = k.  The page gathers the statistic over all MoE layers at
+ * once: pass the layers' logits and idx stacked as T = layers * tokens rows.
+ *   logits [T,E] float (moe_route's logits), idx [T,k] int32 (in)
+ *   mask [T] uint8 or NULL: rows with 0 (padding) are not counted (in)
+ *   aux [1] float (out); f [k,E] float, P [E] float: the statistics, or NULL (out)
+ * Only s.T, s.E and s.k are used (s.d and s.d_ff are ignored).  Deterministic
+ * (fixed reduction order); aux = 0 when no row is counted.
+ */
+int moe_aux_loss(moe_shape s, const float* logits, const int32_t* idx, const uint8_t* mask,
+                 float* aux, float* f, float* P, void* stream);
 
 /*
  * moe_forward_static -- moe_forward for callers that cannot allocate device

@@ -30,7 +30,7 @@ EXPORTS = (
     "moe_forward_workspace_bytes", "moe_forward_hostio_workspace_bytes", "moe_route",
     "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_stall_test", "moe_combine",
     "moe_forward", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_static",
-    "moe_read_device_status",
+    "moe_aux_loss", "moe_block_workspace_bytes", "moe_block_forward", "moe_read_device_status",
 )
 
 MOE_STATIC_SCRATCH_BYTES = 8 << 20
@@ -67,7 +67,7 @@ def lib() -> ctypes.CDLL:
         L.moe_check_shape.restype = I
         L.moe_check_shape.argtypes = [S]
         for fn in ("moe_expert_workspace_bytes", "moe_forward_workspace_bytes",
-                   "moe_forward_hostio_workspace_bytes"):
+                   "moe_forward_hostio_workspace_bytes", "moe_block_workspace_bytes"):
             getattr(L, fn).restype = Z
             getattr(L, fn).argtypes = [S]
         L.moe_route.restype = I
@@ -89,6 +89,10 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_hostio.argtypes = [S, P, P, P, P, P, P, P, P, Z, P]
         L.moe_forward_static.restype = I
         L.moe_forward_static.argtypes = [S, P, P, P, P, P, P, P, P, P]
+        L.moe_block_forward.restype = I
+        L.moe_block_forward.argtypes = [S, P, P, ctypes.c_float, P, P, P, P, P, P, P, Z, P]
+        L.moe_aux_loss.restype = I
+        L.moe_aux_loss.argtypes = [S, P, P, P, P, P, P, P]
         L.moe_read_device_status.restype = I
         L.moe_read_device_status.argtypes = [P, P]
         _lib = L
@@ -331,6 +335,47 @@ def moe_forward_static(shape, x, Wg, bias, W1, W3, W2, y=None, device_status=Non
            lib().moe_forward_static(_shape(shape), _p(x), _p(Wg), _p(bias), _p(W1), _p(W3),
                                     _p(W2), _p(y), _p(device_status), _stream(stream)))
     return y
+
+
+def moe_block_workspace_bytes(shape) -> int:
+    return lib().moe_block_workspace_bytes(_shape(shape))
+
+
+def moe_block_forward(shape, U, gamma, Wg, bias, W1, W3, W2, eps=1e-5, H=None, ws=None,
+                      stream=None):
+    """H = U + MoE(RMSNorm(U)) through moe_block_forward."""
+    T, d, d_ff, E, k = shape
+    _dev(U, "U", torch.bfloat16, (T, d))
+    _dev(gamma, "gamma", torch.bfloat16, (d,))
+    _dev(Wg, "Wg", torch.bfloat16, (d, E))
+    _dev(bias, "bias", torch.float32, (E,))
+    _dev(W1, "W1", torch.bfloat16, (E, d, d_ff))
+    _dev(W3, "W3", torch.bfloat16, (E, d, d_ff))
+    _dev(W2, "W2", torch.bfloat16, (E, d_ff, d))
+    H = _new((T, d), torch.bfloat16, U) if H is None else H
+    ws = workspace(moe_block_workspace_bytes(shape), U.device) if ws is None else ws
+    _dev(H, "H", torch.bfloat16, (T, d))
+    _dev(ws, "ws", torch.uint8)
+    _check("moe_block_forward",
+           lib().moe_block_forward(_shape(shape), _p(U), _p(gamma), float(eps), _p(Wg), _p(bias),
+                                   _p(W1), _p(W3), _p(W2), _p(H), _p(ws), ws.numel(),
+                                   _stream(stream)))
+    return H
+
+
+def moe_aux_loss(shape, logits, idx, mask=None, want_stats=False, stream=None):
+    """Load-balancing term E * sum_s sum_i f_{s,i} P_i.  Returns (aux [1], f [k,E] or None,
+    P [E] or None) as CUDA float32 tensors.  shape's T is the number of rows of logits."""
+    T, d, d_ff, E, k = shape
+    _dev(logits, "logits", torch.float32, (T, E))
+    _dev(idx, "idx", torch.int32, (T, k))
+    _dev(mask, "mask", torch.uint8, (T,))
+    aux = _new((1,), torch.float32, logits)
+    f = _new((k, E), torch.float32, logits) if want_stats else None
+    P = _new((E,), torch.float32, logits) if want_stats else None
+    _check("moe_aux_loss", lib().moe_aux_loss(_shape(shape), _p(logits), _p(idx), _p(mask), _p(aux),
+                                              _p(f), _p(P), _stream(stream)))
+    return aux, f, P
 
 
 def moe_read_device_status(ws, stream=None) -> int:

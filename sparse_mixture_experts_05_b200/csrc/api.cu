@@ -11,6 +11,8 @@
 #include <cstring>
 #include <mutex>
 
+#include "aux_loss.cuh"
+#include "block.cuh"
 #include "combine.cuh"
 #include "common.cuh"
 #include "dispatch.cuh"
@@ -90,7 +92,8 @@ constexpr int kProfileEvents = 7;
 // GEMM1, 5 after GEMM2, 6 after the combine.
 int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                  const void* W1, const void* W3, const void* W2, void* y, int32_t* idx_out,
-                 float* gate_out, void* ws, cudaStream_t st, void* const* events) {
+                 float* gate_out, void* ws, cudaStream_t st, void* const* events,
+                 const void* residual = nullptr) {
     auto mark = [&](int i) {
         return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
     };
@@ -118,7 +121,7 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
                       events ? events[4] : nullptr);
     if (rc) return rc;
     if (!mark(5)) return MOE_ERR_CUDA;
-    rc = launch_combine(s, o, inv, gate, y, st);
+    rc = launch_combine(s, o, inv, gate, y, st, residual);
     if (rc) return rc;
     return mark(6) ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -175,6 +178,11 @@ size_t moe_expert_workspace_bytes(moe_shape s) {
 size_t moe_forward_workspace_bytes(moe_shape s) {
     if (check_shape(s)) return 0;
     return fwd_layout(s).total;
+}
+
+size_t moe_block_workspace_bytes(moe_shape s) {
+    if (check_shape(s)) return 0;
+    return fwd_layout(s).total + align_up((size_t)s.T * s.d * 2, 256);
 }
 
 size_t moe_forward_hostio_workspace_bytes(moe_shape s) {
@@ -275,6 +283,22 @@ int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float
                         static_cast<cudaStream_t>(stream), events);
 }
 
+int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, const void* Wg,
+                      const float* bias, const void* W1, const void* W3, const void* W2, void* H,
+                      void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(U) || !ok_ptr(gamma) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) ||
+        !ok_ptr(W3) || !ok_ptr(W2) || !ok_ptr(H) || !ok_ptr(ws) || !(eps >= 0.0f))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_block_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void* u = static_cast<char*>(ws) + moe_forward_workspace_bytes(s);
+    rc = launch_rmsnorm(s, U, gamma, eps, u, st);
+    if (rc) return rc;
+    return forward_impl(s, u, Wg, bias, W1, W3, W2, H, nullptr, nullptr, ws, st, nullptr, U);
+}
+
 int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const float* bias,
                        const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
                        size_t ws_bytes, void* stream) {
@@ -319,6 +343,16 @@ int moe_forward_static(moe_shape s, const void* x, const void* Wg, const float* 
             cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+int moe_aux_loss(moe_shape s, const float* logits, const int32_t* idx, const uint8_t* mask,
+                 float* aux, float* f, float* P, void* stream) {
+    // Only T, E and k matter here (T may count the rows of several layers).
+    if (s.T < 0 || s.E < 1 || s.k < 1 || s.k > s.E) return MOE_ERR_INVALID_ARG;
+    if (s.E > 32 || s.k > 8) return MOE_ERR_UNSUPPORTED;
+    if (!ok_ptr(aux) || !ok_opt(f) || !ok_opt(P) || !ok_opt(mask)) return MOE_ERR_INVALID_ARG;
+    if (s.T > 0 && (!ok_ptr(logits) || !ok_ptr(idx))) return MOE_ERR_INVALID_ARG;
+    return launch_aux_loss(s, logits, idx, mask, aux, f, P, static_cast<cudaStream_t>(stream));
 }
 
 int moe_read_device_status(const void* ws, void* stream) {

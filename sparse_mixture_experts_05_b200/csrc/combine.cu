@@ -21,7 +21,8 @@ namespace combine {
 // over the whole GPU instead of one warp per row.
 __global__ void __launch_bounds__(256)
     combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ inv,
-                   const float* __restrict__ gate, int T, int d8, int k, uint4* __restrict__ y) {
+                   const float* __restrict__ gate, int T, int d8, int k,
+                   const uint4* __restrict__ residual, uint4* __restrict__ y) {
     const int64_t total = (int64_t)T * d8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -49,6 +50,15 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
         }
+        if (residual) {  // H = U + MoE(.): one more float32 addition before the rounding
+            const uint4 r = __ldg(residual + i);
+            const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc[2 * j] = __fadd_rn(bf16_lo(w[j]), acc[2 * j]);
+                acc[2 * j + 1] = __fadd_rn(bf16_hi(w[j]), acc[2 * j + 1]);
+            }
+        }
         y[i] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                           pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
     }
@@ -57,14 +67,15 @@ __global__ void __launch_bounds__(256)
 }  // namespace combine
 
 int launch_combine(const moe_shape& s, const float* o, const int32_t* inv, const float* gate,
-                   void* y, cudaStream_t stream) {
+                   void* y, cudaStream_t stream, const void* residual) {
     using namespace combine;
     if (s.T == 0) return MOE_OK;
     const int64_t work = (int64_t)s.T * (s.d / 8);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256,
                                                                  (int64_t)device_sm_count() * 8));
     combine_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(o), inv, gate, s.T,
-                                             s.d / 8, s.k, static_cast<uint4*>(y));
+                                             s.d / 8, s.k, static_cast<const uint4*>(residual),
+                                             static_cast<uint4*>(y));
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -8,8 +8,9 @@
 
 namespace moe {
 
-// y[t] = bf16( sum over slots s, in order, of gate[t,s] * o[inv[t,s]] ).
+// y[t] = bf16( sum over slots s, in order, of gate[t,s] * o[inv[t,s]] ), plus
+// residual[t] (bf16, nullable) added in float32 before the rounding.
 int launch_combine(const moe_shape& s, const float* o, const int32_t* inv, const float* gate,
-                   void* y, cudaStream_t stream);
+                   void* y, cudaStream_t stream, const void* residual = nullptr);
 
 }  // namespace moe

@@ -102,6 +102,17 @@ def test_null_and_misaligned_pointers_are_rejected_without_launch():
                  None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_aux_loss_rejects_bad_arguments_on_host():
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    assert _call("moe_aux_loss", binding.MoeShape(16, 128, 256, 8, 9), good, good, None, good,
+                 None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_aux_loss", binding.MoeShape(16, 128, 256, 8, 2), good, good, None, None,
+                 None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_aux_loss", binding.MoeShape(16, 128, 256, 64, 2), good, good, None, good,
+                 None, None, None) == moe.MOE_ERR_UNSUPPORTED
+
+
 def test_empty_batch_is_a_no_op_on_host():
     S = binding.MoeShape(0, 128, 256, 8, 2)
     for fn, nargs in (("moe_route", 7), ("moe_combine", 5)):
