@@ -17,7 +17,7 @@
 // Roles (192 threads, one CTA per SM):
 //   warp 0      TMA producer: A box [128 x 64] (K-major) + B boxes [64 x 64] (MN-major)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2..5  epilogue: tcgen05.ld -> SiLU(.) / convert -> global stores
+//   warps 2..5  epilogue: tcgen05.ld -> SiLU(.) / convert -> TMA stores of 32 x 32 chunks
 // Shared-memory stages are recycled through full/empty mbarriers; the two TMEM
 // accumulator buffers (2 x 256 columns) let the epilogue of tile i overlap the
 // MMAs of tile i+1.
@@ -58,7 +58,11 @@ constexpr int kAccCols = 256;
 constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kThreads = 192;
 constexpr int kMaxE = 32;
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024;
+constexpr int kEpiBufBytes = 4096;                              // 32 rows x 128 bytes
+constexpr int kEpiWarpBytes = 2 * kEpiBufBytes;                 // two staging buffers
+constexpr int kEpiBytes = 4 * kEpiWarpBytes;                    // four epilogue warps
+constexpr int kOutBox = 32;                                     // output box: 32 x 32
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kEpiBytes + 1024;
 
 struct Params {
     const int32_t* offsets;  // [E+1]
@@ -106,18 +110,56 @@ __device__ __forceinline__ TileInfo decode_tile_rows(int t, const int* mt_prefix
     return ti;
 }
 
+// Epilogue output path.  A warp owns 32 rows of the tile (one TMEM lane quarter)
+// and writes them 32 columns at a time.  When all 32 rows belong to the tile's
+// expert, the chunk is staged in shared memory in the output tensor map's
+// swizzled layout (one row per lane; the swizzle spreads the lanes' 16-byte
+// writes over all banks) and leaves as one TMA store, so global memory sees
+// whole rows instead of 32 scattered 16-byte pieces per instruction.  Each warp
+// alternates between two staging buffers; before refilling one, lane 0 waits
+// until the store issued from it has finished reading shared memory.  Warps
+// whose rows run past the expert (the last tile of each expert) store row by
+// row with predication instead, since a tensor-map store cannot skip rows.
+struct EpiStage {
+    uint8_t* base;  // this warp's two buffers, 1024-byte aligned
+    uint32_t next;  // buffer to fill next
+};
+
+// Hands out the next staging buffer once the store that last read it is done.
+__device__ __forceinline__ uint8_t* epi_acquire(EpiStage& st, int lane) {
+    uint8_t* buf = st.base + st.next * kEpiBufBytes;
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+    return buf;
+}
+
+// Publishes a filled buffer to the TMA unit and stores it at (x, y).
+__device__ __forceinline__ void epi_release(EpiStage& st, const CUtensorMap* map, uint8_t* buf,
+                                            int x, int y, int lane) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map, buf, x, y);
+        bulk_commit_group();
+    }
+    st.next ^= 1u;
+}
+
 // GEMM1 epilogue of one TMEM lane (= one row): columns [0, hcols) hold
 // a = x W1, columns [hcols, 2 hcols) hold b = x W3 for the same output columns;
-// h = SiLU(a) * b = a / (1 + exp(-a)) * b.
-__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, __nv_bfloat16* hrow,
-                                                int hcols) {
+// h = SiLU(a) * b = a / (1 + exp(-a)) * b.  With `tma` the warp's 32 rows go
+// out through `map` (bf16, 64-byte rows, 64-byte swizzle) at (x0 + c, y0).
+__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, bool tma,
+                                                __nv_bfloat16* hrow, int hcols,
+                                                const CUtensorMap* map, EpiStage& st, int x0,
+                                                int y0, int lane) {
 #pragma unroll 1
     for (int c = 0; c < hcols; c += 32) {
         uint32_t ra[32], rb[32];
         tmem_ld_32cols(taddr + c, ra);
         tmem_ld_32cols(taddr + hcols + c, rb);
         tmem_ld_wait();
-        if (valid) {
+        if (valid || tma) {
             uint32_t packed[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -129,24 +171,48 @@ __device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, __nv
                 const float h1 = a1 / (1.0f + __expf(-a1)) * b1;
                 packed[j] = pack_bf16x2(h0, h1);
             }
-            uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+            if (tma) {
+                uint8_t* buf = epi_acquire(st, lane);
+                uint8_t* rowp = buf + lane * 64;
+                const int sw = (lane >> 1) & 3;  // 64-byte swizzle: chunk ^= address bits 7..8
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                    packed[4 * j + 3]);
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
+                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                   packed[4 * j + 3]);
+                epi_release(st, map, buf, x0 + c, y0, lane);
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                        packed[4 * j + 3]);
+            }
         }
     }
 }
 
 // GEMM2 epilogue of one TMEM lane: `ncols` fp32 columns stored as they are.
-__device__ __forceinline__ void epilogue_store_f32(uint32_t taddr, bool valid, float* orow,
-                                                   int ncols) {
+// With `tma` the warp's rows go out through `map` (fp32, 128-byte rows,
+// 128-byte swizzle) at (x0 + c, y0).
+__device__ __forceinline__ void epilogue_store_f32(uint32_t taddr, bool valid, bool tma,
+                                                   float* orow, int ncols, const CUtensorMap* map,
+                                                   EpiStage& st, int x0, int y0, int lane) {
 #pragma unroll 1
     for (int c = 0; c < ncols; c += 32) {
         uint32_t r[32];
         tmem_ld_32cols(taddr + c, r);
         tmem_ld_wait();
-        if (valid) {
+        if (tma) {
+            uint8_t* buf = epi_acquire(st, lane);
+            uint8_t* rowp = buf + lane * 128;
+            const int sw = lane & 7;  // 128-byte swizzle: chunk ^= address bits 7..9
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
+                    make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            epi_release(st, map, buf, x0 + c, y0, lane);
+        } else if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -159,7 +225,8 @@ template <bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB0,
-                       const __grid_constant__ CUtensorMap tmB1, const Params p) {
+                       const __grid_constant__ CUtensorMap tmB1,
+                       const __grid_constant__ CUtensorMap tmOut, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -203,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmB0);
         if (kSwiGLU) tma_prefetch_map(&tmB1);
+        tma_prefetch_map(&tmOut);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_slot, kTmemCols);
@@ -325,6 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------- epilogue (warps 2..5)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int row_in_tile = q * 32 + lane;
+        EpiStage st{smem + kStages * kStageBytes + q * kEpiWarpBytes, 0u};
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
@@ -338,21 +407,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after_sync();
             const uint32_t taddr = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
             const bool valid = row_in_tile < ti.rows;
+            const bool tma = q * 32 + 32 <= ti.rows;  // warp-uniform: all 32 rows are the expert's
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
+            const int y0 = ti.row0 + q * 32;
             if (kSwiGLU)
-                epilogue_swiglu(taddr, valid, reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                                  grow * p.n_out + ti.n0,
-                                p.n_tile_out);
+                epilogue_swiglu(taddr, valid, tma,
+                                reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + ti.n0,
+                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane);
             else
-                epilogue_store_f32(taddr, valid, reinterpret_cast<float*>(p.out) +
-                                                     grow * p.n_out + ti.n0,
-                                   p.n_boxes * kBoxN);
+                epilogue_store_f32(taddr, valid, tma,
+                                   reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0,
+                                   p.n_boxes * kBoxN, &tmOut, st, ti.n0, y0, lane);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        // The staging buffers must outlive every store that reads them.
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     }
 
     tc_fence_before_sync();
@@ -385,14 +459,15 @@ constexpr int kPM = 256;                                       // rows per pair 
 constexpr int kPairStages = 6;
 constexpr int kPairBBoxes = 2;                                 // B boxes per CTA per stage (max)
 constexpr int kPairStageBytes = kABytes + kPairBBoxes * kBBoxBytes;   // 32 KB
-constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + 1024;
+constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + kEpiBytes + 1024;
 constexpr int kPairMinRows = 512;
 
 template <bool kSwiGLU>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB0,
-                            const __grid_constant__ CUtensorMap tmB1, const Params p) {
+                            const __grid_constant__ CUtensorMap tmB1,
+                            const __grid_constant__ CUtensorMap tmOut, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -439,6 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmB0);
         if (kSwiGLU) tma_prefetch_map(&tmB1);
+        tma_prefetch_map(&tmOut);
     }
     if (warp == 1) {
         tmem_alloc_pair(&tmem_slot, kTmemCols);
@@ -566,6 +642,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
         const int row_in_cta = q * 32 + lane;
+        EpiStage st{smem + kPairStages * kPairStageBytes + q * kEpiWarpBytes, 0u};
         int acc = 0;
         uint32_t acc_phase = 0;
         const uint32_t leader_acc_empty0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
@@ -581,21 +658,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t taddr = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
             const int row_in_tile = (int)rank * kBM + row_in_cta;
             const bool valid = row_in_tile < ti.rows;
+            const int warp_row0 = (int)rank * kBM + q * 32;
+            const bool tma = warp_row0 + 32 <= ti.rows;  // warp-uniform
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
+            const int y0 = ti.row0 + warp_row0;
             if (kSwiGLU)
-                epilogue_swiglu(taddr, valid, reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                                  grow * p.n_out + ti.n0,
-                                p.n_tile_out);
+                epilogue_swiglu(taddr, valid, tma,
+                                reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + ti.n0,
+                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane);
             else
-                epilogue_store_f32(taddr, valid, reinterpret_cast<float*>(p.out) +
-                                                     grow * p.n_out + ti.n0,
-                                   2 * boxes * kBoxN);
+                epilogue_store_f32(taddr, valid, tma,
+                                   reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0,
+                                   2 * boxes * kBoxN, &tmOut, st, ti.n0, y0, lane);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * (uint32_t)sizeof(uint64_t));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     }
 
     tc_fence_before_sync();
@@ -645,9 +727,29 @@ static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+// Output map for the epilogue's TMA stores: a row-major [rows, cols] matrix of
+// bf16 (h) or fp32 (o) with a 32 x 32-element box; the box rows are 64 or 128
+// bytes, swizzled in shared memory with the matching 64- or 128-byte pattern.
+static bool make_out_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         bool f32) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t esize = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * esize};
+    cuuint32_t box[2] = {kOutBox, kOutBox};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <bool kSwiGLU>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                  const Params& p, int max_tiles, cudaStream_t stream) {
+                  const CUtensorMap& out, const Params& p, int max_tiles, cudaStream_t stream) {
     auto kern = expert_gemm_kernel<kSwiGLU>;
     static int configured_device = -1;
     int dev = 0;
@@ -659,7 +761,7 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
         configured_device = dev;
     }
     const int grid = max(1, min(device_sm_count(), max_tiles));
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(a, b0, b1, p);
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(a, b0, b1, out, p);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -704,11 +806,13 @@ static int max_pairs() {
 
 template <bool kSwiGLU>
 static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                       const Params& p, int max_tiles, cudaStream_t stream) {
+                       const CUtensorMap& out, const Params& p, int max_tiles,
+                       cudaStream_t stream) {
     const int pairs = max_pairs<kSwiGLU>();  // also sets the shared-memory attribute
     if (pairs <= 0) return MOE_ERR_CUDA;
     const int grid = 2 * max(1, min(pairs, max_tiles));
-    expert_gemm_pair_kernel<kSwiGLU><<<grid, kThreads, kPairSmemBytes, stream>>>(a, b0, b1, p);
+    expert_gemm_pair_kernel<kSwiGLU><<<grid, kThreads, kPairSmemBytes, stream>>>(a, b0, b1, out,
+                                                                                 p);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -721,9 +825,11 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     using namespace gemm;
     const int R = s.T * s.k;
     if (R == 0) return MOE_OK;
-    CUtensorMap mx, mh, m1, m3, m2;
+    CUtensorMap mx, mh, m1, m3, m2, oh, oo;
     if (!make_map(&mx, x_sorted, (uint64_t)R, (uint64_t)s.d, kBM) ||
         !make_map(&mh, h, (uint64_t)R, (uint64_t)s.d_ff, kBM) ||
+        !make_out_map(&oh, h, (uint64_t)R, (uint64_t)s.d_ff, false) ||
+        !make_out_map(&oo, o, (uint64_t)R, (uint64_t)s.d, true) ||
         !make_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
         !make_map(&m3, W3, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
         !make_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, kBK))
@@ -760,8 +866,8 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.stall_after = stall_after;
     p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
     const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / p1.n_tile_out);
-    int rc = pairs1 ? launch_pair<true>(mx, m1, m3, p1, t1, stream)
-                    : launch<true>(mx, m1, m3, p1, t1, stream);
+    int rc = pairs1 ? launch_pair<true>(mx, m1, m3, oh, p1, t1, stream)
+                    : launch<true>(mx, m1, m3, oh, p1, t1, stream);
     if (rc != MOE_OK) return rc;
     if (mid_event && cudaEventRecord(static_cast<cudaEvent_t>(mid_event), stream) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -775,8 +881,8 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.stall_after = stall_after;
     p2.group_m = group_rows(pairs2 ? kPM : kBM, s.d_ff);
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
-    return pairs2 ? launch_pair<false>(mh, m2, m2, p2, t2, stream)
-                  : launch<false>(mh, m2, m2, p2, t2, stream);
+    return pairs2 ? launch_pair<false>(mh, m2, m2, oo, p2, t2, stream)
+                  : launch<false>(mh, m2, m2, oo, p2, t2, stream);
 }
 
 }  // namespace moe
