@@ -61,12 +61,19 @@ def _load():
         lib.orc_gather.argtypes = [I, I, P, P, P]
         lib.orc_expert.restype = I
         lib.orc_expert.argtypes = [I, I, I, I, P, P, P, P, P, I, P, P]
+        lib.orc_expert_bias.restype = I
+        lib.orc_expert_bias.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, I, P, P]
         lib.orc_combine.restype = None
         lib.orc_combine.argtypes = [I, I, I, P, P, P, P]
         lib.orc_forward.restype = I
         lib.orc_forward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, P]
         lib.orc_forward_tokens.restype = I
         lib.orc_forward_tokens.argtypes = [I, P, I, I, I, I, I, P, P, P, P, P, P, I, P, P, P]
+        lib.orc_forward_bias.restype = I
+        lib.orc_forward_bias.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, I, P, P, P]
+        lib.orc_forward_tokens_bias.restype = I
+        lib.orc_forward_tokens_bias.argtypes = [I, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, I,
+                                                P, P, P]
         lib.orc_rmsnorm.restype = None
         lib.orc_rmsnorm.argtypes = [I, I, P, P, ctypes.c_double, P]
         lib.orc_block_forward.restype = I
@@ -152,9 +159,19 @@ def gather(x, perm_tok):
     return out
 
 
-def expert(x_sorted, offsets, W1, W3, W2, round_h: bool = True):
+def _expert_bias(expert_bias, E: int, d: int, d_ff: int):
+    """(b1 [E,d_ff], b3 [E,d_ff], b2 [E,d]) as float32 arrays, or three Nones."""
+    if expert_bias is None:
+        return None, None, None
+    b1, b3, b2 = (np.ascontiguousarray(b, dtype=np.float32) for b in expert_bias)
+    assert b1.shape == (E, d_ff) and b3.shape == (E, d_ff) and b2.shape == (E, d)
+    return b1, b3, b2
+
+
+def expert(x_sorted, offsets, W1, W3, W2, round_h: bool = True, expert_bias=None):
     """SwiGLU experts over sorted rows.  Returns (h [R,d_ff], o [R,d]) as float64 values
-    (h rounded to bf16 values when round_h; o never rounded)."""
+    (h rounded to bf16 values when round_h; o never rounded).  expert_bias =
+    (b1, b3, b2) adds the biases of the three Linear layers."""
     xs = _u16(x_sorted)
     W1 = _u16(W1)
     W3 = _u16(W3)
@@ -163,10 +180,11 @@ def expert(x_sorted, offsets, W1, W3, W2, round_h: bool = True):
     R, d = xs.shape
     E, d1, d_ff = W1.shape
     assert d1 == d and W3.shape == W1.shape and W2.shape == (E, d_ff, d)
+    b1, b3, b2 = _expert_bias(expert_bias, E, d, d_ff)
     h = np.empty((R, d_ff), np.float64)
     o = np.empty((R, d), np.float64)
-    rc = _load().orc_expert(R, d, d_ff, E, _p(offsets), _p(xs), _p(W1), _p(W3), _p(W2),
-                            int(round_h), _p(h), _p(o))
+    rc = _load().orc_expert_bias(R, d, d_ff, E, _p(offsets), _p(xs), _p(W1), _p(W3), _p(W2),
+                                 _p(b1), _p(b3), _p(b2), int(round_h), _p(h), _p(o))
     if rc:
         raise ValueError(f"orc_expert failed (rc={rc})")
     return h, o
@@ -183,8 +201,9 @@ def combine(o, inv, gate):
     return y
 
 
-def forward(x, wg, W1, W3, W2, k: int, bias=None, round_h: bool = True):
-    """Whole layer, expert-major.  Returns (y float64 [T,d] unrounded, idx [T,k], gate [T,k])."""
+def forward(x, wg, W1, W3, W2, k: int, bias=None, round_h: bool = True, expert_bias=None):
+    """Whole layer, expert-major.  Returns (y float64 [T,d] unrounded, idx [T,k], gate [T,k]).
+    bias: router bias [E]; expert_bias: (b1, b3, b2) of the expert Linear layers."""
     x = _u16(x)
     wg = _u16(wg)
     W1 = _u16(W1)
@@ -196,14 +215,16 @@ def forward(x, wg, W1, W3, W2, k: int, bias=None, round_h: bool = True):
     idx = np.empty((T, k), np.int32)
     gate = np.empty((T, k), np.float32)
     b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
-    rc = _load().orc_forward(T, d, d_ff, E, k, _p(x), _p(wg), _p(b), _p(W1), _p(W3), _p(W2),
-                             int(round_h), _p(y), _p(idx), _p(gate))
+    b1, b3, b2 = _expert_bias(expert_bias, E, d, d_ff)
+    rc = _load().orc_forward_bias(T, d, d_ff, E, k, _p(x), _p(wg), _p(b), _p(W1), _p(W3), _p(W2),
+                                  _p(b1), _p(b3), _p(b2), int(round_h), _p(y), _p(idx), _p(gate))
     if rc:
         raise ValueError(f"orc_forward failed (rc={rc})")
     return y, idx, gate
 
 
-def forward_tokens(tokens, x, wg, W1, W3, W2, k: int, bias=None, round_h: bool = True):
+def forward_tokens(tokens, x, wg, W1, W3, W2, k: int, bias=None, round_h: bool = True,
+                   expert_bias=None):
     """Naive per-token loop for the listed tokens.  Returns (y [n,d], idx [n,k], gate [n,k])."""
     toks = np.ascontiguousarray(tokens, dtype=np.int32)
     x = _u16(x)
@@ -218,8 +239,10 @@ def forward_tokens(tokens, x, wg, W1, W3, W2, k: int, bias=None, round_h: bool =
     idx = np.empty((n, k), np.int32)
     gate = np.empty((n, k), np.float32)
     b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
-    rc = _load().orc_forward_tokens(n, _p(toks), T, d, d_ff, E, k, _p(x), _p(wg), _p(b), _p(W1),
-                                    _p(W3), _p(W2), int(round_h), _p(y), _p(idx), _p(gate))
+    b1, b3, b2 = _expert_bias(expert_bias, E, d, d_ff)
+    rc = _load().orc_forward_tokens_bias(n, _p(toks), T, d, d_ff, E, k, _p(x), _p(wg), _p(b),
+                                         _p(W1), _p(W3), _p(W2), _p(b1), _p(b3), _p(b2),
+                                         int(round_h), _p(y), _p(idx), _p(gate))
     if rc:
         raise ValueError(f"orc_forward_tokens failed (rc={rc})")
     return y, idx, gate

@@ -159,10 +159,14 @@ void orc_gather(int R, int d, const int32_t* perm_tok, const uint16_t* x, uint16
  * Section "Прямой проход в формулах": (SiLU(u W_gate) * (u W_up)) W_down with
  * W_gate = W1[e], W_up = W3[e] of shape [d, d_ff] and W_down = W2[e] of shape
  * [d_ff, d], all row-major.  h [d_ff] holds the bf16-rounded value (round_h) or
- * the unrounded one; o [d] is unrounded.
+ * the unrounded one; o [d] is unrounded.  b1e/b3e [d_ff] and b2e [d] are the
+ * float biases of the three Linear layers when the layer is built with bias
+ * (section "Подсчёт параметров", teaching configuration: bias on every Linear),
+ * else NULL.
  * acc_a / acc_b are caller scratch of d_ff doubles. */
 static void expert_row(int d, int d_ff, const uint16_t* u, const uint16_t* W1e,
-                       const uint16_t* W3e, const uint16_t* W2e, int round_h,
+                       const uint16_t* W3e, const uint16_t* W2e, const float* b1e,
+                       const float* b3e, const float* b2e, int round_h,
                        double* acc_a, double* acc_b, double* h, double* o) {
     for (int n = 0; n < d_ff; ++n) { acc_a[n] = 0.0; acc_b[n] = 0.0; }
     /* a_n = sum_j u_j W1[j][n], b_n = sum_j u_j W3[j][n]; each sum runs over j
@@ -176,26 +180,31 @@ static void expert_row(int d, int d_ff, const uint16_t* u, const uint16_t* W1e,
             acc_b[n] += uj * orc_bf16_value(w3[n]);
         }
     }
+    /* Linear layers with bias (the teaching configuration) add b after the sum. */
+    if (b1e) for (int n = 0; n < d_ff; ++n) acc_a[n] += (double)b1e[n];
+    if (b3e) for (int n = 0; n < d_ff; ++n) acc_b[n] += (double)b3e[n];
     for (int n = 0; n < d_ff; ++n) {
         double hv = orc_silu(acc_a[n]) * acc_b[n];
         h[n] = round_h ? orc_round_bf16(hv) : hv;
     }
-    /* o_c = sum_n h_n W2[n][c], n ascending. */
+    /* o_c = sum_n h_n W2[n][c], n ascending (+ b2_c). */
     for (int c = 0; c < d; ++c) o[c] = 0.0;
     for (int n = 0; n < d_ff; ++n) {
         double hn = h[n];
         const uint16_t* w2 = W2e + (int64_t)n * d;
         for (int c = 0; c < d; ++c) o[c] += hn * orc_bf16_value(w2[c]);
     }
+    if (b2e) for (int c = 0; c < d; ++c) o[c] += (double)b2e[c];
 }
 
 /* Expert_e(X[tok]) for every expert over its sorted rows (section "Алгоритм";
  * an expert with no rows is not called).
  *   x_sorted [R, d] bf16, offsets [E+1], W1/W3 [E, d, d_ff], W2 [E, d_ff, d]
  *   h [R, d_ff] double, o [R, d] double. */
-int orc_expert(int R, int d, int d_ff, int E, const int32_t* offsets, const uint16_t* x_sorted,
-               const uint16_t* W1, const uint16_t* W3, const uint16_t* W2, int round_h,
-               double* h, double* o) {
+int orc_expert_bias(int R, int d, int d_ff, int E, const int32_t* offsets,
+                    const uint16_t* x_sorted, const uint16_t* W1, const uint16_t* W3,
+                    const uint16_t* W2, const float* b1, const float* b3, const float* b2,
+                    int round_h, double* h, double* o) {
     if (offsets[0] != 0 || offsets[E] != R) return 1;
     for (int e = 0; e < E; ++e)
         if (offsets[e + 1] < offsets[e]) return 1;
@@ -214,14 +223,22 @@ int orc_expert(int R, int d, int d_ff, int E, const int32_t* offsets, const uint
                 while (offsets[e + 1] <= r) ++e;
                 const int64_t wsz = (int64_t)d * d_ff;
                 expert_row(d, d_ff, x_sorted + (int64_t)r * d, W1 + e * wsz, W3 + e * wsz,
-                           W2 + e * wsz, round_h, acc_a, acc_b, h + (int64_t)r * d_ff,
-                           o + (int64_t)r * d);
+                           W2 + e * wsz, b1 ? b1 + (int64_t)e * d_ff : NULL,
+                           b3 ? b3 + (int64_t)e * d_ff : NULL, b2 ? b2 + (int64_t)e * d : NULL,
+                           round_h, acc_a, acc_b, h + (int64_t)r * d_ff, o + (int64_t)r * d);
             }
         }
         free(acc_a);
         free(acc_b);
     }
     return ok ? 0 : 2;
+}
+
+int orc_expert(int R, int d, int d_ff, int E, const int32_t* offsets, const uint16_t* x_sorted,
+               const uint16_t* W1, const uint16_t* W3, const uint16_t* W2, int round_h,
+               double* h, double* o) {
+    return orc_expert_bias(R, d, d_ff, E, offsets, x_sorted, W1, W3, W2, NULL, NULL, NULL,
+                           round_h, h, o);
 }
 
 /* ---- combine ------------------------------------------------------------------
@@ -243,9 +260,10 @@ void orc_combine(int T, int d, int k, const double* o, const int32_t* inv, const
 /* ---- whole layer, expert-major (the loop of section "Алгоритм") ------------
  * Scratch is allocated here; outputs idx/gate/offsets/perm_tok/inv are
  * nullable. */
-int orc_forward(int T, int d, int d_ff, int E, int k, const uint16_t* x, const uint16_t* wg,
-                const float* bias, const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
-                int round_h, double* y, int32_t* idx_out, float* gate_out) {
+int orc_forward_bias(int T, int d, int d_ff, int E, int k, const uint16_t* x, const uint16_t* wg,
+                     const float* bias, const uint16_t* W1, const uint16_t* W3,
+                     const uint16_t* W2, const float* b1, const float* b3, const float* b2,
+                     int round_h, double* y, int32_t* idx_out, float* gate_out) {
     const int R = T * k;
     int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)(R > 0 ? R : 1));
     float* gate = (float*)malloc(sizeof(float) * (size_t)(R > 0 ? R : 1));
@@ -260,7 +278,8 @@ int orc_forward(int T, int d, int d_ff, int E, int k, const uint16_t* x, const u
     if ((rc = orc_route(T, d, E, k, x, wg, bias, idx, gate, NULL))) goto done;
     if ((rc = orc_dispatch(T, E, k, idx, offsets, perm, inv))) goto done;
     orc_gather(R, d, perm, x, xs);
-    if ((rc = orc_expert(R, d, d_ff, E, offsets, xs, W1, W3, W2, round_h, h, o))) goto done;
+    if ((rc = orc_expert_bias(R, d, d_ff, E, offsets, xs, W1, W3, W2, b1, b3, b2, round_h, h, o)))
+        goto done;
     orc_combine(T, d, k, o, inv, gate, y);
     if (idx_out) memcpy(idx_out, idx, sizeof(int32_t) * (size_t)R);
     if (gate_out) memcpy(gate_out, gate, sizeof(float) * (size_t)R);
@@ -269,16 +288,24 @@ done:
     return rc;
 }
 
+int orc_forward(int T, int d, int d_ff, int E, int k, const uint16_t* x, const uint16_t* wg,
+                const float* bias, const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
+                int round_h, double* y, int32_t* idx_out, float* gate_out) {
+    return orc_forward_bias(T, d, d_ff, E, k, x, wg, bias, W1, W3, W2, NULL, NULL, NULL, round_h,
+                            y, idx_out, gate_out);
+}
+
 /* ---- naive per-token loop ------------------------------------------------------
  * The same layer computed token by token, straight from the formula of section
  * "Прямой проход в формулах" (the reference's own test compares MoE against such
  * a loop, section "Алгоритм").  Computes y only for the n listed tokens:
  *   toks [n] token ids; y [n, d] double; idx_out [n, k], gate_out [n, k]
  * (nullable).  Used for sampled checks at sizes where the full layer is too slow. */
-int orc_forward_tokens(int n, const int32_t* toks, int T, int d, int d_ff, int E, int k,
-                       const uint16_t* x, const uint16_t* wg, const float* bias,
-                       const uint16_t* W1, const uint16_t* W3, const uint16_t* W2, int round_h,
-                       double* y, int32_t* idx_out, float* gate_out) {
+int orc_forward_tokens_bias(int n, const int32_t* toks, int T, int d, int d_ff, int E, int k,
+                            const uint16_t* x, const uint16_t* wg, const float* bias,
+                            const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
+                            const float* b1, const float* b3, const float* b2, int round_h,
+                            double* y, int32_t* idx_out, float* gate_out) {
     if (E < 1 || E > 64 || k < 1 || k > E) return 1;
     for (int i = 0; i < n; ++i)
         if (toks[i] < 0 || toks[i] >= T) return 1;
@@ -300,9 +327,13 @@ int orc_forward_tokens(int n, const int32_t* toks, int T, int d, int d_ff, int E
                 float w[64];
                 route_one(d, E, k, u, wg, bias, sel, w, NULL);
                 const int64_t wsz = (int64_t)d * d_ff;
-                for (int s = 0; s < k; ++s)
-                    expert_row(d, d_ff, u, W1 + sel[s] * wsz, W3 + sel[s] * wsz, W2 + sel[s] * wsz,
+                for (int s = 0; s < k; ++s) {
+                    const int e = sel[s];
+                    expert_row(d, d_ff, u, W1 + e * wsz, W3 + e * wsz, W2 + e * wsz,
+                               b1 ? b1 + (int64_t)e * d_ff : NULL,
+                               b3 ? b3 + (int64_t)e * d_ff : NULL, b2 ? b2 + (int64_t)e * d : NULL,
                                round_h, acc_a, acc_b, h, o + (int64_t)s * d);
+                }
                 for (int c = 0; c < d; ++c) {
                     double acc = 0.0;
                     for (int s = 0; s < k; ++s) acc += (double)w[s] * o[(int64_t)s * d + c];
@@ -315,6 +346,14 @@ int orc_forward_tokens(int n, const int32_t* toks, int T, int d, int d_ff, int E
         free(acc_a); free(acc_b); free(h); free(o);
     }
     return ok ? 0 : 2;
+}
+
+int orc_forward_tokens(int n, const int32_t* toks, int T, int d, int d_ff, int E, int k,
+                       const uint16_t* x, const uint16_t* wg, const float* bias,
+                       const uint16_t* W1, const uint16_t* W3, const uint16_t* W2, int round_h,
+                       double* y, int32_t* idx_out, float* gate_out) {
+    return orc_forward_tokens_bias(n, toks, T, d, d_ff, E, k, x, wg, bias, W1, W3, W2, NULL, NULL,
+                                   NULL, round_h, y, idx_out, gate_out);
 }
 
 /* ---- parameter count ------------------------------------------------------------

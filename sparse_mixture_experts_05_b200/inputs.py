@@ -86,6 +86,24 @@ def make_inputs(T: int, d: int, d_ff: int, E: int, k: int, seed: int, bias: bool
     return out
 
 
+def expert_biases(E: int, d: int, d_ff: int, seed: int, device: str = "cpu"):
+    """Biases of the three expert Linear layers for the layer built with bias
+    (the teaching configuration of the Mixtral page's section "Подсчёт
+    параметров"): b1, b3 [E, d_ff] ~ U(-1/sqrt(d), 1/sqrt(d)) and b2 [E, d] ~
+    U(-1/sqrt(d_ff), 1/sqrt(d_ff)) (the usual Linear initialisation), rounded to
+    bf16 values and held as float32.  Drawn from their own generator, seeded
+    with `seed`, in the order b1, b3, b2."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+
+    def uni(shape, bound):
+        t = torch.rand(*shape, generator=gen, device=device, dtype=torch.float32)
+        return (t * (2 * bound) - bound).to(torch.bfloat16).to(torch.float32)
+
+    return (uni((E, d_ff), 1.0 / math.sqrt(d)), uni((E, d_ff), 1.0 / math.sqrt(d)),
+            uni((E, d), 1.0 / math.sqrt(d_ff)))
+
+
 def workload_inputs(name: str, device: str = "cpu", T: int | None = None) -> dict:
     """Inputs of a named workload; `T` overrides the token count (same seed)."""
     w = WORKLOADS[name]

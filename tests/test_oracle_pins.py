@@ -20,7 +20,7 @@ import torch
 from scipy.special import expit
 
 import oracle
-from sparse_mixture_experts_05_b200.inputs import identical_experts, make_inputs
+from sparse_mixture_experts_05_b200.inputs import expert_biases, identical_experts, make_inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -344,6 +344,95 @@ def test_planted_mistakes_fail_the_pins():
     W2t = sq["W2"].transpose(1, 2).contiguous()
     y_t, _, _ = oracle.forward(sq["x"], sq["Wg"], sq["W1"], sq["W3"], W2t, 1, round_h=False)
     assert np.max(np.abs(y_t - ref_sq)) > 1e-3 * np.max(np.abs(ref_sq))
+
+
+# ---------------------------------------------------------------- expert Linear biases
+# The teaching configuration of the Mixtral page (section "Подсчёт параметров",
+# bias on every Linear) gives each expert's three projections a bias:
+# SwiGLU(u) = (SiLU(u W1 + b1) * (u W3 + b3)) W2 + b2.
+
+def _dense_swiglu_bias(x, W1, W3, W2, b1, b3, b2):
+    a = x @ W1 + b1
+    b = x @ W3 + b3
+    return ((a * expit(a)) * b) @ W2 + b2
+
+
+def _np_bias(bs):
+    return tuple(b.numpy().astype(np.float64) for b in bs)
+
+
+def test_expert_bias_E1_k1_reduces_to_dense_linear_layers_with_bias():
+    inp = make_inputs(40, 64, 96, 1, 1, seed=13)
+    eb = expert_biases(1, 64, 96, seed=113)
+    y, _, _ = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], 1,
+                             round_h=False, expert_bias=eb)
+    b1, b3, b2 = _np_bias(eb)
+    ref = _dense_swiglu_bias(_f64(inp["x"]), _f64(inp["W1"][0]), _f64(inp["W3"][0]),
+                             _f64(inp["W2"][0]), b1[0], b3[0], b2[0])
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+    # and the biases matter: without them the result is far off
+    y0, _, _ = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], 1,
+                              round_h=False)
+    assert np.max(np.abs(y0 - ref)) > 1e-3 * np.max(np.abs(ref))
+
+
+def test_expert_bias_closed_forms_with_zero_weights():
+    """W2 = 0: every expert returns b2[e], so y_t = sum_s gate_ts b2[idx_ts].
+    W1 = W3 = 0: h = SiLU(b1[e]) * b3[e] for every row of expert e."""
+    T, d, d_ff, E, k = 30, 64, 96, 8, 2
+    inp = make_inputs(T, d, d_ff, E, k, seed=14)
+    eb = expert_biases(E, d, d_ff, seed=114)
+    b1, b3, b2 = _np_bias(eb)
+    zW2 = torch.zeros_like(inp["W2"])
+    y, idx, gate = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], zW2, k,
+                                  round_h=False, expert_bias=eb)
+    ref = np.einsum("ts,tsc->tc", gate.astype(np.float64), b2[idx])
+    assert np.max(np.abs(y - ref)) <= 1e-15 * np.max(np.abs(ref))
+    zW = torch.zeros_like(inp["W1"])
+    offsets = np.array([0, 3, 3, 7, 8, 8, 8, 12, 15], np.int32)
+    xs = inp["x"][:15]
+    h, o = oracle.expert(xs, offsets, zW, zW, inp["W2"], round_h=False, expert_bias=eb)
+    row_e = np.repeat(np.arange(E), np.diff(offsets))
+    h_ref = (b1 * expit(b1) * b3)[row_e]
+    assert np.max(np.abs(h - h_ref)) <= 1e-15 * np.max(np.abs(h_ref))
+    o_ref = np.stack([h_ref[r] @ _f64(inp["W2"][row_e[r]]) + b2[row_e[r]] for r in range(15)])
+    assert np.max(np.abs(o - o_ref)) <= 1e-12 * np.max(np.abs(o_ref))
+
+
+def test_expert_bias_layer_equals_dense_all_experts_masked():
+    T, d, d_ff, E, k = 60, 64, 96, 8, 2
+    inp = make_inputs(T, d, d_ff, E, k, seed=15, bias=True)
+    eb = expert_biases(E, d, d_ff, seed=115)
+    b1, b3, b2 = _np_bias(eb)
+    y, _, _ = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k,
+                             bias=inp["bias"], round_h=False, expert_bias=eb)
+    x = _f64(inp["x"])
+    g = _logits_numpy(inp).astype(np.float32).astype(np.float64)
+    order = np.lexsort((np.tile(np.arange(E), (T, 1)), -g), axis=1)[:, :k]
+    p = np.exp(g - g.max(1, keepdims=True))
+    G = np.zeros_like(p)
+    np.put_along_axis(G, order, np.take_along_axis(p, order, 1), 1)
+    G /= G.sum(1, keepdims=True)
+    ref = np.zeros_like(x)
+    for e in range(E):
+        ref += G[:, e:e + 1] * _dense_swiglu_bias(x, _f64(inp["W1"][e]), _f64(inp["W3"][e]),
+                                                  _f64(inp["W2"][e]), b1[e], b3[e], b2[e])
+    assert np.max(np.abs(y - ref)) <= 2e-6 * np.max(np.abs(ref))
+    # swapping the gate and up biases must break the pin
+    ys, _, _ = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k,
+                              bias=inp["bias"], round_h=False, expert_bias=(eb[1], eb[0], eb[2]))
+    assert np.max(np.abs(ys - ref)) > 1e-3 * np.max(np.abs(ref))
+
+
+def test_expert_bias_per_token_loop_equals_expert_major_loop():
+    inp = make_inputs(50, 64, 160, 8, 2, seed=16)
+    eb = expert_biases(8, 64, 160, seed=116)
+    y, idx, gate = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], 2,
+                                  expert_bias=eb)
+    toks = np.arange(50)[::-1].copy()
+    y2, idx2, _ = oracle.forward_tokens(toks, inp["x"], inp["Wg"], inp["W1"], inp["W3"],
+                                        inp["W2"], 2, expert_bias=eb)
+    assert np.array_equal(y[toks], y2) and np.array_equal(idx[toks], idx2)
 
 
 # ---------------------------------------------------------------- load-balancing loss
