@@ -125,6 +125,21 @@ int moe_expert_swiglu(moe_shape s, const void* x_sorted, const int32_t* offsets,
                       size_t ws_bytes, void* stream);
 
 /*
+ * moe_expert_swiglu_bias -- moe_expert_swiglu for the layer built with bias on
+ * its Linear layers (Mixtral textbook page, section "Подсчёт параметров": the
+ * teaching configuration puts a bias on every Linear):
+ *     h = SiLU(x W1_e + b1_e) (.) (x W3_e + b3_e),   o = h W2_e + b2_e
+ *   b1, b3 [E,d_ff] float, b2 [E,d] float (in; each may be NULL = no bias)
+ * The biases are added in float32 to the float32 accumulators, before SiLU and
+ * the product (b1, b3) and before o is stored (b2).  Everything else as for
+ * moe_expert_swiglu.
+ */
+int moe_expert_swiglu_bias(moe_shape s, const void* x_sorted, const int32_t* offsets,
+                           const void* W1, const void* W3, const void* W2, const float* b1,
+                           const float* b3, const float* b2, void* h, float* o, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
  * moe_expert_swiglu_stall_test -- test hook for the error path of the bounded
  * device waits (no counterpart on the pages).  Runs moe_expert_swiglu with its
  * TMA producer stopping after `stall_after` (>= 0) pipeline stages, as if it had
@@ -158,6 +173,16 @@ int moe_combine(moe_shape s, const float* o, const int32_t* inv, const float* ga
 int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, const void* W1,
                 const void* W3, const void* W2, void* y, int32_t* idx_out, float* gate_out,
                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_forward_bias -- moe_forward with the biases of the expert Linear layers
+ * (b1, b3 [E,d_ff], b2 [E,d] float, each nullable; see moe_expert_swiglu_bias).
+ * The router bias is `bias`, as for moe_forward.
+ */
+int moe_forward_bias(moe_shape s, const void* x, const void* Wg, const float* bias,
+                     const void* W1, const void* W3, const void* W2, const float* b1,
+                     const float* b3, const float* b2, void* y, int32_t* idx_out,
+                     float* gate_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_forward_profiled -- moe_forward (no idx/gate copies) that also records

@@ -7,9 +7,10 @@ Build the library with `python -m sparse_mixture_experts_05_b200.build`.
 """
 from .binding import (  # noqa: F401
     EXPORTS, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED,
-    MOE_ERR_WORKSPACE, MOE_OK, MoeError, moe_check_shape, moe_combine, moe_dispatch,
-    moe_expert_swiglu, moe_expert_swiglu_stall_test, moe_expert_workspace_bytes, moe_forward,
-    moe_forward_hostio, moe_forward_hostio_workspace_bytes, moe_forward_profiled,
-    moe_forward_static, moe_aux_loss, moe_block_forward, moe_block_workspace_bytes, moe_forward_workspace_bytes,
+    MOE_ERR_WORKSPACE, MOE_OK, MoeError, moe_aux_loss, moe_block_forward,
+    moe_block_workspace_bytes, moe_check_shape, moe_combine, moe_dispatch, moe_expert_swiglu,
+    moe_expert_swiglu_bias, moe_expert_swiglu_stall_test, moe_expert_workspace_bytes, moe_forward,
+    moe_forward_bias, moe_forward_hostio, moe_forward_hostio_workspace_bytes,
+    moe_forward_profiled, moe_forward_static, moe_forward_workspace_bytes,
     moe_read_device_status, moe_route, status_string, workspace,
 )

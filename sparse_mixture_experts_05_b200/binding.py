@@ -28,8 +28,8 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 EXPORTS = (
     "moe_status_string", "moe_check_shape", "moe_expert_workspace_bytes",
     "moe_forward_workspace_bytes", "moe_forward_hostio_workspace_bytes", "moe_route",
-    "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_stall_test", "moe_combine",
-    "moe_forward", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_static",
+    "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_bias", "moe_expert_swiglu_stall_test",
+    "moe_combine", "moe_forward", "moe_forward_bias", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_static",
     "moe_aux_loss", "moe_block_workspace_bytes", "moe_block_forward", "moe_read_device_status",
 )
 
@@ -80,6 +80,10 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_swiglu_stall_test.argtypes = [S, P, P, P, P, P, P, P, P, Z, I,
                                                    ctypes.c_uint64, P]
         L.moe_combine.restype = I
+        L.moe_expert_swiglu_bias.restype = I
+        L.moe_expert_swiglu_bias.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, Z, P]
+        L.moe_forward_bias.restype = I
+        L.moe_forward_bias.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, Z, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P]
         L.moe_forward.restype = I
         L.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, Z, P]
@@ -224,6 +228,30 @@ def moe_expert_swiglu(shape, x_sorted, offsets, W1, W3, W2, h=None, o=None, ws=N
     return h, o, ws
 
 
+def _expert_bias_args(shape, expert_bias):
+    """(b1, b3, b2) float32 device tensors [E,d_ff], [E,d_ff], [E,d], each may be None."""
+    T, d, d_ff, E, k = shape
+    if expert_bias is None:
+        return None, None, None
+    b1, b3, b2 = expert_bias
+    _dev(b1, "b1", torch.float32, (E, d_ff))
+    _dev(b3, "b3", torch.float32, (E, d_ff))
+    _dev(b2, "b2", torch.float32, (E, d))
+    return b1, b3, b2
+
+
+def moe_expert_swiglu_bias(shape, x_sorted, offsets, W1, W3, W2, expert_bias, h=None, o=None,
+                           ws=None, stream=None):
+    """moe_expert_swiglu with the expert Linear biases expert_bias = (b1, b3, b2)."""
+    h, o, ws = _expert_args(shape, x_sorted, offsets, W1, W3, W2, h, o, ws)
+    b1, b3, b2 = _expert_bias_args(shape, expert_bias)
+    _check("moe_expert_swiglu_bias",
+           lib().moe_expert_swiglu_bias(_shape(shape), _p(x_sorted), _p(offsets), _p(W1), _p(W3),
+                                        _p(W2), _p(b1), _p(b3), _p(b2), _p(h), _p(o), _p(ws),
+                                        ws.numel(), _stream(stream)))
+    return h, o, ws
+
+
 def moe_expert_swiglu_stall_test(shape, x_sorted, offsets, W1, W3, W2, stall_after: int,
                                  timeout_ns: int, h=None, o=None, ws=None, stream=None):
     h, o, ws = _expert_args(shape, x_sorted, offsets, W1, W3, W2, h, o, ws)
@@ -265,6 +293,30 @@ def moe_forward(shape, x, Wg, bias, W1, W3, W2, y=None, idx_out=None, gate_out=N
     _check("moe_forward", lib().moe_forward(_shape(shape), _p(x), _p(Wg), _p(bias), _p(W1), _p(W3),
                                             _p(W2), _p(y), _p(idx_out), _p(gate_out), _p(ws),
                                             ws.numel(), _stream(stream)))
+    return y
+
+
+def moe_forward_bias(shape, x, Wg, bias, W1, W3, W2, expert_bias, y=None, idx_out=None,
+                     gate_out=None, ws=None, stream=None):
+    """moe_forward with the expert Linear biases expert_bias = (b1, b3, b2)."""
+    T, d, d_ff, E, k = shape
+    _dev(x, "x", torch.bfloat16, (T, d))
+    _dev(Wg, "Wg", torch.bfloat16, (d, E))
+    _dev(bias, "bias", torch.float32, (E,))
+    _dev(W1, "W1", torch.bfloat16, (E, d, d_ff))
+    _dev(W3, "W3", torch.bfloat16, (E, d, d_ff))
+    _dev(W2, "W2", torch.bfloat16, (E, d_ff, d))
+    b1, b3, b2 = _expert_bias_args(shape, expert_bias)
+    y = _new((T, d), torch.bfloat16, x) if y is None else y
+    ws = workspace(moe_forward_workspace_bytes(shape), x.device) if ws is None else ws
+    _dev(y, "y", torch.bfloat16, (T, d))
+    _dev(idx_out, "idx_out", torch.int32, (T, k))
+    _dev(gate_out, "gate_out", torch.float32, (T, k))
+    _dev(ws, "ws", torch.uint8)
+    _check("moe_forward_bias",
+           lib().moe_forward_bias(_shape(shape), _p(x), _p(Wg), _p(bias), _p(W1), _p(W3), _p(W2),
+                                  _p(b1), _p(b3), _p(b2), _p(y), _p(idx_out), _p(gate_out),
+                                  _p(ws), ws.numel(), _stream(stream)))
     return y
 
 

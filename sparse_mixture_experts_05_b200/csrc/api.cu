@@ -90,10 +90,17 @@ constexpr int kProfileEvents = 7;
 // Records events[i] (when given) between the launches: 0 before the router, 1
 // after it, 2 after the dispatch index kernel, 3 after the scatter, 4 after
 // GEMM1, 5 after GEMM2, 6 after the combine.
+// Biases of the expert Linear layers (each nullable): b1, b3 [E, d_ff], b2 [E, d].
+struct ExpertBias {
+    const float* b1 = nullptr;
+    const float* b3 = nullptr;
+    const float* b2 = nullptr;
+};
+
 int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                  const void* W1, const void* W3, const void* W2, void* y, int32_t* idx_out,
                  float* gate_out, void* ws, cudaStream_t st, void* const* events,
-                 const void* residual = nullptr) {
+                 const void* residual = nullptr, const ExpertBias& eb = ExpertBias{}) {
     auto mark = [&](int i) {
         return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
     };
@@ -118,7 +125,7 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     if (rc) return rc;
     if (!mark(3)) return MOE_ERR_CUDA;
     rc = expert_gemms(s, xs, offsets, W1, W3, W2, h, o, status, kDefaultWaitTimeoutNs, -1, st,
-                      events ? events[4] : nullptr);
+                      events ? events[4] : nullptr, eb.b1, eb.b3, eb.b2);
     if (rc) return rc;
     if (!mark(5)) return MOE_ERR_CUDA;
     rc = launch_combine(s, o, inv, gate, y, st, residual);
@@ -230,6 +237,22 @@ int moe_expert_swiglu(moe_shape s, const void* x_sorted, const int32_t* offsets,
                         kDefaultWaitTimeoutNs, -1, st, nullptr);
 }
 
+int moe_expert_swiglu_bias(moe_shape s, const void* x_sorted, const int32_t* offsets,
+                           const void* W1, const void* W3, const void* W2, const float* b1,
+                           const float* b3, const float* b2, void* h, float* o, void* ws,
+                           size_t ws_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x_sorted) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_opt(b1) || !ok_opt(b3) || !ok_opt(b2) || !ok_ptr(h) || !ok_ptr(o) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_expert_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return MOE_ERR_CUDA;
+    return expert_gemms(s, x_sorted, offsets, W1, W3, W2, h, o, static_cast<int*>(ws),
+                        kDefaultWaitTimeoutNs, -1, st, nullptr, b1, b3, b2);
+}
+
 int moe_expert_swiglu_stall_test(moe_shape s, const void* x_sorted, const int32_t* offsets,
                                  const void* W1, const void* W3, const void* W2, void* h, float* o,
                                  void* ws, size_t ws_bytes, int stall_after,
@@ -266,6 +289,25 @@ int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, c
     if (ws_bytes < moe_forward_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
     return forward_impl(s, x, Wg, bias, W1, W3, W2, y, idx_out, gate_out, ws,
                         static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int moe_forward_bias(moe_shape s, const void* x, const void* Wg, const float* bias,
+                     const void* W1, const void* W3, const void* W2, const float* b1,
+                     const float* b3, const float* b2, void* y, int32_t* idx_out,
+                     float* gate_out, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_opt(b1) || !ok_opt(b3) || !ok_opt(b2) || !ok_ptr(y) || !ok_opt(idx_out) ||
+        !ok_opt(gate_out) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    ExpertBias eb;
+    eb.b1 = b1;
+    eb.b3 = b3;
+    eb.b2 = b2;
+    return forward_impl(s, x, Wg, bias, W1, W3, W2, y, idx_out, gate_out, ws,
+                        static_cast<cudaStream_t>(stream), nullptr, nullptr, eb);
 }
 
 int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float* bias,

@@ -76,6 +76,8 @@ struct Params {
     int n_boxes;             // B boxes per stage (MMA N = 64 * n_boxes)
     int stall_after;         // test hook: producer stops after this many stages (-1: never)
     int group_m;             // m-tiles per rasterisation group (see decode_tile_rows)
+    const float* bias_a;     // GEMM1: b1 [E, n_out]; GEMM2: b2 [E, n_out]; or nullptr
+    const float* bias_b;     // GEMM1: b3 [E, n_out]; or nullptr
 };
 
 struct TileInfo {
@@ -145,20 +147,39 @@ __device__ __forceinline__ void epi_release(EpiStage& st, const CUtensorMap* map
     st.next ^= 1u;
 }
 
+// r[j] += bias[j] for 32 consecutive float32 columns (the same for every lane:
+// the loads are broadcasts).  Float32 addition, as the bias of a Linear layer
+// is added to its float32 accumulator.
+__device__ __forceinline__ void add_bias_32(uint32_t (&r)[32], const float* bias) {
+    const float4* b4 = reinterpret_cast<const float4*>(bias);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 b = __ldg(b4 + j);
+        r[4 * j + 0] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 0]), b.x));
+        r[4 * j + 1] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 1]), b.y));
+        r[4 * j + 2] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 2]), b.z));
+        r[4 * j + 3] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 3]), b.w));
+    }
+}
+
 // GEMM1 epilogue of one TMEM lane (= one row): columns [0, hcols) hold
 // a = x W1, columns [hcols, 2 hcols) hold b = x W3 for the same output columns;
 // h = SiLU(a) * b = a / (1 + exp(-a)) * b.  With `tma` the warp's 32 rows go
 // out through `map` (bf16, 64-byte rows, 64-byte swizzle) at (x0 + c, y0).
+// ba / bb (nullable) are the biases of the tile's first column for a and b.
 __device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, bool tma,
                                                 __nv_bfloat16* hrow, int hcols,
                                                 const CUtensorMap* map, EpiStage& st, int x0,
-                                                int y0, int lane) {
+                                                int y0, int lane, const float* ba,
+                                                const float* bb) {
 #pragma unroll 1
     for (int c = 0; c < hcols; c += 32) {
         uint32_t ra[32], rb[32];
         tmem_ld_32cols(taddr + c, ra);
         tmem_ld_32cols(taddr + hcols + c, rb);
         tmem_ld_wait();
+        if (ba) add_bias_32(ra, ba + c);
+        if (bb) add_bias_32(rb, bb + c);
         if (valid || tma) {
             uint32_t packed[16];
 #pragma unroll
@@ -192,17 +213,20 @@ __device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, bool
     }
 }
 
-// GEMM2 epilogue of one TMEM lane: `ncols` fp32 columns stored as they are.
-// With `tma` the warp's rows go out through `map` (fp32, 128-byte rows,
-// 128-byte swizzle) at (x0 + c, y0).
+// GEMM2 epilogue of one TMEM lane: `ncols` fp32 columns stored as they are
+// (plus the bias `bo` of the tile's first column, when given).  With `tma` the
+// warp's rows go out through `map` (fp32, 128-byte rows, 128-byte swizzle) at
+// (x0 + c, y0).
 __device__ __forceinline__ void epilogue_store_f32(uint32_t taddr, bool valid, bool tma,
                                                    float* orow, int ncols, const CUtensorMap* map,
-                                                   EpiStage& st, int x0, int y0, int lane) {
+                                                   EpiStage& st, int x0, int y0, int lane,
+                                                   const float* bo) {
 #pragma unroll 1
     for (int c = 0; c < ncols; c += 32) {
         uint32_t r[32];
         tmem_ld_32cols(taddr + c, r);
         tmem_ld_wait();
+        if (bo) add_bias_32(r, bo + c);
         if (tma) {
             uint8_t* buf = epi_acquire(st, lane);
             uint8_t* rowp = buf + lane * 128;
@@ -410,14 +434,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool tma = q * 32 + 32 <= ti.rows;  // warp-uniform: all 32 rows are the expert's
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
             const int y0 = ti.row0 + q * 32;
+            const int64_t boff = (int64_t)ti.e * p.n_out + ti.n0;
+            const float* ba = p.bias_a ? p.bias_a + boff : nullptr;
+            const float* bb = p.bias_b ? p.bias_b + boff : nullptr;
             if (kSwiGLU)
                 epilogue_swiglu(taddr, valid, tma,
                                 reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + ti.n0,
-                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane);
+                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane, ba, bb);
             else
                 epilogue_store_f32(taddr, valid, tma,
                                    reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0,
-                                   p.n_boxes * kBoxN, &tmOut, st, ti.n0, y0, lane);
+                                   p.n_boxes * kBoxN, &tmOut, st, ti.n0, y0, lane, ba);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -662,14 +689,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool tma = warp_row0 + 32 <= ti.rows;  // warp-uniform
             const int64_t grow = (int64_t)ti.row0 + row_in_tile;
             const int y0 = ti.row0 + warp_row0;
+            const int64_t boff = (int64_t)ti.e * p.n_out + ti.n0;
+            const float* ba = p.bias_a ? p.bias_a + boff : nullptr;
+            const float* bb = p.bias_b ? p.bias_b + boff : nullptr;
             if (kSwiGLU)
                 epilogue_swiglu(taddr, valid, tma,
                                 reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + ti.n0,
-                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane);
+                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane, ba, bb);
             else
                 epilogue_store_f32(taddr, valid, tma,
                                    reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0,
-                                   2 * boxes * kBoxN, &tmOut, st, ti.n0, y0, lane);
+                                   2 * boxes * kBoxN, &tmOut, st, ti.n0, y0, lane, ba);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * (uint32_t)sizeof(uint64_t));
@@ -821,7 +851,7 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
 int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offsets, const void* W1,
                  const void* W3, const void* W2, void* h, float* o, int* err,
                  uint64_t timeout_ns, int stall_after, cudaStream_t stream,
-                 void* mid_event) {
+                 void* mid_event, const float* b1, const float* b3, const float* b2) {
     using namespace gemm;
     const int R = s.T * s.k;
     if (R == 0) return MOE_OK;
@@ -865,6 +895,8 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.n_boxes = pairs1 ? 2 : 4;  // per CTA
     p1.stall_after = stall_after;
     p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
+    p1.bias_a = b1;
+    p1.bias_b = b3;
     const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / p1.n_tile_out);
     int rc = pairs1 ? launch_pair<true>(mx, m1, m3, oh, p1, t1, stream)
                     : launch<true>(mx, m1, m3, oh, p1, t1, stream);
@@ -880,6 +912,8 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.n_boxes = p2.n_tile_out / kBoxN / (pairs2 ? 2 : 1);
     p2.stall_after = stall_after;
     p2.group_m = group_rows(pairs2 ? kPM : kBM, s.d_ff);
+    p2.bias_a = b2;
+    p2.bias_b = nullptr;
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
     return pairs2 ? launch_pair<false>(mh, m2, m2, oo, p2, t2, stream)
                   : launch<false>(mh, m2, m2, oo, p2, t2, stream);

@@ -96,7 +96,7 @@ def _silu_parts(a):
     return a * sig, sig * (1.0 + a * (1.0 - sig))
 
 
-def check_expert_rows(hv, ov, xv, row_expert, W1, W3, W2, h_ref, o_ref):
+def check_expert_rows(hv, ov, xv, row_expert, W1, W3, W2, h_ref, o_ref, expert_bias=None):
     """Expert kernel outputs on the given sorted rows against the oracle, with
     a-priori float32 accumulation bounds.
 
@@ -108,9 +108,13 @@ def check_expert_rows(hv, ov, xv, row_expert, W1, W3, W2, h_ref, o_ref):
     |error| <= (K/16 + 16) * 2^-24 * sum|terms|.  h = SiLU(a) * b is then within
     one bf16 ulp of the oracle's bf16 h plus the propagated accumulation error;
     o differs from the oracle's o by at most |h - h_ref| . |W2| plus GEMM2's own
-    accumulation error.  Returns (fraction of h elements that differ, max o
-    error / its bound).
+    accumulation error.  With expert_bias = (b1, b3, b2) (float32 tensors) each
+    bias is one more float32 addition: 2^-24 of the sum's magnitude on a, b and
+    o.  Returns (fraction of h elements that differ, max o error / its bound).
     """
+    u = 2.0 ** -24
+    if expert_bias is not None:
+        b1s, b3s, b2s = (b.detach().cpu().numpy().astype(np.float64) for b in expert_bias)
     from_bf16 = bf16_values
     K1 = xv.shape[1]
     K2 = hv.shape[1]
@@ -127,6 +131,11 @@ def check_expert_rows(hv, ov, xv, row_expert, W1, W3, W2, h_ref, o_ref):
         b = x @ w3
         sa = np.abs(x) @ np.abs(w1)
         sb = np.abs(x) @ np.abs(w3)
+        if expert_bias is not None:
+            a = a + b1s[int(e)]
+            b = b + b3s[int(e)]
+            sa = sa + np.abs(a) / g1 * u     # the bias addition's rounding, in units of g1
+            sb = sb + np.abs(b) / g1 * u
         silu, dsilu = _silu_parts(a)
         # + float32 evaluation of SiLU(a) * b itself (a few float32 ulps of h)
         tol_h = (bf16_ulp(h_ref[m]) * 1.0001 + g1 * (np.abs(dsilu * b) * sa + np.abs(silu) * sb)
@@ -134,6 +143,8 @@ def check_expert_rows(hv, ov, xv, row_expert, W1, W3, W2, h_ref, o_ref):
         dh = np.abs(hv[m] - h_ref[m])
         assert np.all(dh <= tol_h), float(np.max(dh / tol_h))
         tol_o = dh @ np.abs(w2) + g2 * (np.abs(hv[m]) @ np.abs(w2))
+        if expert_bias is not None:
+            tol_o = tol_o + u * (np.abs(o_ref[m]) + tol_o)
         do = np.abs(ov[m] - o_ref[m])
         assert np.all(do <= tol_o * 1.0001 + 1e-30), float(np.max(do / (tol_o + 1e-30)))
         worst = max(worst, float(np.max(do / (tol_o + 1e-30))))

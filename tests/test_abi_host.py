@@ -100,6 +100,15 @@ def test_null_and_misaligned_pointers_are_rejected_without_launch():
     assert _call("moe_expert_swiglu_stall_test", S, good, good, good, good, good, good, good,
                  good, ctypes.c_size_t(1 << 20), -1, ctypes.c_uint64(10 ** 6),
                  None) == moe.MOE_ERR_INVALID_ARG
+    # biased variants: a misaligned bias, then a short workspace
+    assert _call("moe_expert_swiglu_bias", S, good, good, good, good, good, good, bad, None,
+                 good, good, good, ctypes.c_size_t(1 << 20), None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_expert_swiglu_bias", S, good, good, good, good, good, None, None, None,
+                 good, good, good, ctypes.c_size_t(16), None) == moe.MOE_ERR_WORKSPACE
+    assert _call("moe_forward_bias", S, good, good, None, good, good, good, bad, good, good, good,
+                 None, None, good, ctypes.c_size_t(1 << 30), None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_forward_bias", S, good, good, None, good, good, good, good, good, good, good,
+                 None, None, good, ctypes.c_size_t(16), None) == moe.MOE_ERR_WORKSPACE
 
 
 def test_aux_loss_rejects_bad_arguments_on_host():
