@@ -264,33 +264,50 @@ def time_workload(name, steps, warmup, device, rank, tokens=None, experts=None):
     moe.moe_forward(shape, x, Wg, bias, W1, W3, W2, y=y, idx_out=idx, ws=ws)
     counts = torch.bincount(idx.flatten().long(), minlength=w.E).tolist()
 
+    plain = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(steps)]
+
+    def run_plain(i):
+        plain[i][0].record()
+        moe.moe_forward(shape, x, Wg, bias, W1, W3, W2, y=y, ws=ws)
+        plain[i][1].record()
+
     return dict(inp=inp, shape=shape, ws=ws, y=y, flush=flush, events=events, counts=counts,
+                plain=plain, run_plain=run_plain,
                 run=lambda i: moe.moe_forward_profiled(shape, x, Wg, bias, W1, W3, W2, events[i],
                                                        y=y, ws=ws))
 
 
-def timed_loop(ctx, steps, pg, device, clock):
+def timed_loop(ctx, steps, pg, device, clock, profiled):
+    """K timed steps, L2 flushed before each.  profiled=False: each step is one
+    moe_forward between two events (the step time).  profiled=True: each step is
+    moe_forward_profiled, whose seven events split the step by kernel."""
     import torch
     barrier(pg, device)
     torch.cuda.synchronize()
-    clock.start()
+    if clock is not None:
+        clock.start()
     outer0 = torch.cuda.Event(enable_timing=True)
     outer1 = torch.cuda.Event(enable_timing=True)
     outer0.record()
+    run = ctx["run"] if profiled else ctx["run_plain"]
     for i in range(steps):
         ctx["flush"].fill_(i & 0xFF)
-        ctx["run"](i)
+        run(i)
     outer1.record()
     torch.cuda.synchronize()
     barrier(pg, device)
-    clocks = clock.stop()
-    ev = ctx["events"]
-    step_ms = [ev[i][0].elapsed_time(ev[i][6]) for i in range(steps)]
+    clocks = clock.stop() if clock is not None else None
     parts = {}
-    import sparse_mixture_experts_05_b200 as moe
-    names = moe.binding.PROFILE_EVENTS
-    for j in range(1, len(names)):
-        parts[names[j]] = sum(ev[i][j - 1].elapsed_time(ev[i][j]) for i in range(steps)) / steps
+    if profiled:
+        import sparse_mixture_experts_05_b200 as moe
+        ev = ctx["events"]
+        step_ms = [ev[i][0].elapsed_time(ev[i][6]) for i in range(steps)]
+        names = moe.binding.PROFILE_EVENTS
+        for j in range(1, len(names)):
+            parts[names[j]] = sum(ev[i][j - 1].elapsed_time(ev[i][j]) for i in range(steps)) / steps
+    else:
+        step_ms = [a.elapsed_time(b) for a, b in ctx["plain"]]
     return step_ms, parts, outer0.elapsed_time(outer1), clocks
 
 
@@ -363,9 +380,13 @@ def run_ours(a):
 
     ctx = time_workload(a.workload, a.steps, a.warmup, device, rank, a.tokens, a.experts)
     clock = ClockSampler(local)
-    step_ms, parts, bracket_ms, clocks = timed_loop(ctx, a.steps, pg, device, clock)
+    step_ms, _, bracket_ms, clocks = timed_loop(ctx, a.steps, pg, device, clock, profiled=False)
     mean_ms = statistics.mean(step_ms)
     max_ms = reduce_max(pg, mean_ms, device)
+    # the per-kernel split (and the roofline's kernel time) from a second timed
+    # pass of the same steps through moe_forward_profiled
+    p_ms, parts, _, _ = timed_loop(ctx, a.steps, pg, device, None, profiled=True)
+    p_max_ms = reduce_max(pg, statistics.mean(p_ms), device)
     shape = ctx["shape"]
     T = shape[0]
     alg = algorithmic(shape, ctx["counts"])
@@ -416,6 +437,10 @@ def run_ours(a):
         "gpu_launches": 6 * a.steps,
         "clocks": clocks,
         "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
+        "ms_per_step_profiled": round(p_max_ms, 4),
+        "timing": ("value and ms_per_step: moe_forward between two CUDA events per step; "
+                   "kernel_ms, ms_per_step_profiled and the roofline: a second timed pass of "
+                   "the same steps through moe_forward_profiled (events between the launches)"),
         "tflops_layer": round(alg["flops_total"] / (max_ms / 1000) / 1e12, 1),
         "bracket_ms_incl_flush": round(bracket_ms, 3),
     }
@@ -424,8 +449,11 @@ def run_ours(a):
 
     if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
         dctx = time_workload("decode", a.steps, a.warmup, device, rank)
-        d_ms, d_parts, _, d_clocks = timed_loop(dctx, a.steps, pg, device, ClockSampler(local))
+        d_ms, _, _, d_clocks = timed_loop(dctx, a.steps, pg, device, ClockSampler(local),
+                                          profiled=False)
         d_mean = reduce_max(pg, statistics.mean(d_ms), device)
+        d_pms, d_parts, _, _ = timed_loop(dctx, a.steps, pg, device, None, profiled=True)
+        d_pmean = reduce_max(pg, statistics.mean(d_pms), device)
         d_alg = algorithmic(dctx["shape"], dctx["counts"])
         d_gemm = d_parts["gemm1_swiglu"] + d_parts["gemm2_down"]
         d_gbs = d_alg["bytes_experts_decode"] / (d_gemm / 1000) / 1e9
@@ -437,6 +465,7 @@ def run_ours(a):
             "layer_gbs": round((d_alg["bytes_experts_decode"] + d_alg["bytes_router"]) /
                                (d_mean / 1000) / 1e9, 1),
             "kernel_ms": {k_: round(v, 4) for k_, v in d_parts.items()},
+            "ms_per_step_profiled": round(d_pmean, 4),
             "expert_rows": dctx["counts"], "clocks": d_clocks}
         del dctx
         torch.cuda.empty_cache()

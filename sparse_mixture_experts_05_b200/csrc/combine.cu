@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ inv,
                    const float* __restrict__ gate, int T, int d8, int k,
                    const uint4* __restrict__ residual, uint4* __restrict__ y) {
+    grid_dependency_wait();
     const int64_t total = (int64_t)T * d8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -73,10 +74,11 @@ int launch_combine(const moe_shape& s, const float* o, const int32_t* inv, const
     const int64_t work = (int64_t)s.T * (s.d / 8);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256,
                                                                  (int64_t)device_sm_count() * 8));
-    combine_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(o), inv, gate, s.T,
-                                             s.d / 8, s.k, static_cast<const uint4*>(residual),
-                                             static_cast<uint4*>(y));
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, stream,
+                      reinterpret_cast<const float4*>(o), inv, gate, s.T, s.d / 8, s.k,
+                      static_cast<const uint4*>(residual), static_cast<uint4*>(y)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

@@ -44,4 +44,38 @@ int device_sm_count();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Programmatic dependent launch.  The layer's kernels are launched with
+// programmatic stream serialisation: a kernel's CTAs may be scheduled as the
+// previous kernel's CTAs exit, and run their prologue (barrier set-up,
+// tensor-memory allocation, descriptor prefetch) during its tail.  Every such
+// kernel calls grid_dependency_wait() unconditionally, before it reads anything
+// the previous kernel wrote and before any early exit: it returns once the
+// previous grid has completed and its memory operations are visible, so
+// completion of a kernel still implies completion of everything before it in
+// the stream.  Launched without the attribute, the wait returns at once.  No
+// kernel triggers its dependents early (griddepcontrol.launch_dependents):
+// waiting CTAs of the next kernel then sat on the SMs during the whole launch,
+// which measured slower at T = 4096.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// kernel<<<grid, block, smem, stream>>>(args...) with programmatic stream
+// serialisation allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace moe

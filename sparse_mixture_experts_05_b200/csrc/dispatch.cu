@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
+    grid_dependency_wait();
     if (status_to_clear && tid == 0) *status_to_clear = 0;
 
     const int per = (T + kIndexThreads - 1) / kIndexThreads;
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
 __global__ void __launch_bounds__(256)
     scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv, int T, int chunks,
                    int k, uint4* __restrict__ x_sorted) {
+    grid_dependency_wait();
     const int64_t total = (int64_t)T * chunks;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -123,9 +125,10 @@ int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offse
     if (cudaFuncSetAttribute(index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return MOE_ERR_CUDA;
-    index_kernel<<<1, kIndexThreads, smem, stream>>>(idx, s.T, s.E, s.k, offsets, perm_tok, inv,
-                                                     status_to_clear);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(index_kernel, dim3(1), dim3(kIndexThreads), smem, stream, idx, s.T, s.E, s.k,
+                      offsets, perm_tok, inv, status_to_clear) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 int launch_dispatch_scatter(const moe_shape& s, const void* x, const int32_t* inv, void* x_sorted,
@@ -135,9 +138,11 @@ int launch_dispatch_scatter(const moe_shape& s, const void* x, const int32_t* in
     const int64_t work = (int64_t)s.T * (s.d / 8);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256,
                                                                  (int64_t)device_sm_count() * 8));
-    scatter_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(x), inv, s.T, s.d / 8, s.k,
-                                             static_cast<uint4*>(x_sorted));
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(scatter_kernel, dim3(grid), dim3(256), 0, stream,
+                      static_cast<const uint4*>(x), inv, s.T, s.d / 8, s.k,
+                      static_cast<uint4*>(x_sorted)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

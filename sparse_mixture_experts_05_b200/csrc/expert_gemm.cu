@@ -280,15 +280,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&drain_bar, 1);
         fence_barrier_init();
         s_abort = 0;
-        // m-tile prefix over experts (E <= 32, serial)
-        int acc = 0;
-        s_mt[0] = 0;
-        for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
-        for (int e = 0; e < p.E; ++e) {
-            const int cnt = max(0, s_off[e + 1] - s_off[e]);
-            acc += (cnt + kBM - 1) / kBM;
-            s_mt[e + 1] = acc;
-        }
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&tmA);
@@ -299,6 +290,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tmem_alloc(&tmem_slot, kTmemCols);
         tmem_relinquish();
+    }
+    // The set-up above overlaps the previous kernel's tail; the offsets and the
+    // A rows are its output.
+    grid_dependency_wait();
+    if (threadIdx.x == 0) {
+        // m-tile prefix over experts (E <= 32, serial)
+        int acc = 0;
+        s_mt[0] = 0;
+        for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+        for (int e = 0; e < p.E; ++e) {
+            const int cnt = max(0, s_off[e + 1] - s_off[e]);
+            acc += (cnt + kBM - 1) / kBM;
+            s_mt[e + 1] = acc;
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -528,14 +533,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&drain_bar, 1);
         fence_barrier_init();
         s_abort = 0;
-        int acc = 0;
-        s_mt[0] = 0;
-        for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
-        for (int e = 0; e < p.E; ++e) {
-            const int cnt = max(0, s_off[e + 1] - s_off[e]);
-            acc += (cnt + kPM - 1) / kPM;
-            s_mt[e + 1] = acc;
-        }
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&tmA);
@@ -546,6 +543,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tmem_alloc_pair(&tmem_slot, kTmemCols);
         tmem_relinquish_pair();
+    }
+    grid_dependency_wait();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        s_mt[0] = 0;
+        for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+        for (int e = 0; e < p.E; ++e) {
+            const int cnt = max(0, s_off[e + 1] - s_off[e]);
+            acc += (cnt + kPM - 1) / kPM;
+            s_mt[e + 1] = acc;
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -791,8 +799,10 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
         configured_device = dev;
     }
     const int grid = max(1, min(device_sm_count(), max_tiles));
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(a, b0, b1, out, p);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes, stream, a, b0, b1, out, p) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 // Number of CTA pairs that can be resident at once (clusters must fit inside a
@@ -841,9 +851,10 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
     const int pairs = max_pairs<kSwiGLU>();  // also sets the shared-memory attribute
     if (pairs <= 0) return MOE_ERR_CUDA;
     const int grid = 2 * max(1, min(pairs, max_tiles));
-    expert_gemm_pair_kernel<kSwiGLU><<<grid, kThreads, kPairSmemBytes, stream>>>(a, b0, b1, out,
-                                                                                 p);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(expert_gemm_pair_kernel<kSwiGLU>, dim3(grid), dim3(kThreads),
+                      kPairSmemBytes, stream, a, b0, b1, out, p) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 }  // namespace gemm

@@ -59,24 +59,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kSlots = kWarps / KSPLIT;  // token tiles of 16 per block iteration
     extern __shared__ uint4 s_wg[];  // [d/32][NT][32 lanes] x 8 bf16
     __shared__ float s_red[kSlots][KSPLIT][NT][32][4];
+    grid_dependency_wait();
 
     // Stage W_r in fragment order: entry (kb, nt, lane) holds
-    // Wg[kb*32 + (lane&3)*8 + j][nt*8 + (lane>>2)] for j = 0..7 (zero for n >= E).
-    const int nblk = d / 32;
-    for (int i = threadIdx.x; i < nblk * NT * 32; i += blockDim.x) {
-        const int ln = i & 31;
-        const int nt = (i >> 5) % NT;
-        const int kb = i / (32 * NT);
-        const int n = nt * 8 + (ln >> 2);
-        const int k0 = kb * 32 + (ln & 3) * 8;
-        uint32_t w[4];
+    // Wg[kb*32 + (lane&3)*8 + j][nt*8 + (lane>>2)] for j = 0..7 (zero for n >= E),
+    // i.e. element (r, n) goes to half-word r % 8 of entry
+    // (r / 32, n / 8, (n % 8) * 4 + (r % 32) / 8).  Each thread reads whole rows
+    // of W_r (16-byte loads when a row is a multiple of 16 bytes) and scatters
+    // their elements; a warp's 32 consecutive rows land in one 64-byte span per
+    // column, so the 2-byte shared stores do not conflict.
+    uint16_t* s_half = reinterpret_cast<uint16_t*>(s_wg);
+    auto put = [&](int r, int n, uint16_t v) {
+        const int entry = ((r >> 5) * NT + (n >> 3)) * 32 + (n & 7) * 4 + ((r & 31) >> 3);
+        s_half[entry * 8 + (r & 7)] = v;
+    };
+    if ((E & 7) == 0) {
+        const int vec = E >> 3;  // 16-byte pieces per row
+#pragma unroll 4
+        for (int r = threadIdx.x; r < d; r += blockDim.x) {
+            const uint4* row = reinterpret_cast<const uint4*>(wg + (int64_t)r * E);
+            for (int q = 0; q < vec; ++q) {
+                const uint4 v = __ldg(row + q);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t lo = n < E ? wg[(int64_t)(k0 + 2 * j) * E + n] : 0u;
-            const uint32_t hi = n < E ? wg[(int64_t)(k0 + 2 * j + 1) * E + n] : 0u;
-            w[j] = lo | (hi << 16);
+                for (int h = 0; h < 4; ++h) {
+                    put(r, q * 8 + 2 * h, (uint16_t)(w[h] & 0xFFFFu));
+                    put(r, q * 8 + 2 * h + 1, (uint16_t)(w[h] >> 16));
+                }
+            }
         }
-        s_wg[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        for (int r = threadIdx.x; r < d; r += blockDim.x)
+            for (int n = 0; n < NT * 8; ++n)
+                put(r, n, n < E ? __ldg(wg + (int64_t)r * E + n) : (uint16_t)0);
     }
     __syncthreads();
 
@@ -233,8 +248,10 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
-        kern<<<grid, kThreads, smem, stream>>>(xp, wp, bias, s.T, s.d, s.E, s.k, idx, gate, logits);
-        return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+        return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, xp, wp, bias, s.T, s.d,
+                          s.E, s.k, idx, gate, logits) == cudaSuccess
+                   ? MOE_OK
+                   : MOE_ERR_CUDA;
     };
 #define MOE_ROUTER_CASE(N)                                                  \
     case N:                                                                 \

@@ -28,6 +28,8 @@ CASES = {
     "E16k4": (96, 256, 256, 16, 4, 9, False),
     "E5k3": (33, 128, 256, 5, 3, 10, False),
     "single": (1, 128, 256, 8, 2, 11, False),
+    "batch16": (16, 256, 384, 8, 2, 16, True),    # decode-sized: R = 32 rows over 8 experts
+    "batch30": (30, 128, 512, 8, 2, 17, False),
 }
 
 
@@ -215,7 +217,7 @@ def test_forward_deterministic_and_hostio_matches():
     assert torch.equal(y1.cpu(), y_host)
 
 
-@pytest.mark.parametrize("T", [64, 300], ids=["single-cta", "cta-pair"])
+@pytest.mark.parametrize("T", [8, 64, 300], ids=["tiny-batch", "single-cta", "cta-pair"])
 def test_bounded_wait_reports_timeout_and_context_survives(T):
     inp = make_inputs(T, 128, 256, 8, 2, seed=44)
     T, d, d_ff, E, k = inp["shape"]
