@@ -44,7 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 KERNEL_SOURCES = ["sparse_mixture_experts_05_b200/csrc/expert_gemm.cu",
-                  "sparse_mixture_experts_05_b200/csrc/sm100.cuh"]
+                  "sparse_mixture_experts_05_b200/csrc/sm100.cuh",
+                  "sparse_mixture_experts_05_b200/csrc/common.cuh"]
 
 
 def parse(argv=None):
