@@ -80,6 +80,31 @@ struct Params {
     const float* bias_b;     // GEMM1: b3 [E, n_out]; or nullptr
 };
 
+// Tiles are dealt round-robin to `active` workers (CTAs, or CTA pairs): the
+// fewest that still need no more rounds than all `launched` workers would, so
+// every active worker gets the same number of tiles (+-1) and no final round
+// runs a few tiles on a few SMs while the rest idle.  A worker at or beyond
+// `active` gets no tile (first tile = total).
+struct TileDeal {
+    int first, stride;
+};
+__device__ __forceinline__ TileDeal deal_tiles(int worker, int launched, int total) {
+    const int rounds = (total + launched - 1) / launched;
+    const int active = rounds > 0 ? (total + rounds - 1) / rounds : 0;
+    TileDeal d;
+    d.first = worker < active ? worker : total;
+    d.stride = active > 0 ? active : 1;
+    return d;
+}
+
+// Per-stage wait: when the phase completes within try_wait's own suspend window
+// the abort flag is not read; otherwise a bounded wait, then the flag.
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                           volatile int& abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait(bar, parity, timeout_ns) && !abort_flag;
+}
+
 struct TileInfo {
     int e, row0, rows, n0;
 };
@@ -313,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = p.n_out / p.n_tile_out;
     const int total_tiles = s_mt[p.E] * n_tiles;
     const int kb_count = p.K / kBK;
+    const TileDeal deal = deal_tiles(blockIdx.x, gridDim.x, total_tiles);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -323,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued = 0;
             bool ok = true;
             const uint32_t tx_bytes = kABytes + p.n_boxes * kBBoxBytes;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = deal.first; t < total_tiles && ok; t += deal.stride) {
                 const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM, p.group_m);
                 const int wrow0 = ti.e * p.K;
                 for (int kb = 0; kb < kb_count; ++kb) {
@@ -331,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;  // test hook: behave like a producer that died
                         break;
                     }
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns) || s_abort) {
+                    if (!stage_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
                         record_error(p.err, kDeviceTimeoutBase | kRoleProducer);
                         ok = false;
                         break;
@@ -379,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = deal.first; t < total_tiles && ok; t += deal.stride) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns) || s_abort) {
                     record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                     ok = false;
@@ -388,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * kAccCols;
                 for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!mbar_wait(&full_bar[stage], phase, p.timeout_ns) || s_abort) {
+                    if (!stage_wait(&full_bar[stage], phase, p.timeout_ns, s_abort)) {
                         record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                         ok = false;
                         break;
@@ -425,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         EpiStage st{smem + kStages * kStageBytes + q * kEpiWarpBytes, 0u};
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        for (int t = deal.first; t < total_tiles; t += deal.stride) {
             const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kBM, p.group_m);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
@@ -565,6 +591,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int total_tiles = s_mt[p.E] * n_tiles;
     const int kb_count = p.K / kBK;
     const int boxes = p.n_boxes;  // B boxes per CTA per stage
+    const TileDeal deal = deal_tiles(pair, npairs, total_tiles);  // same for both CTAs
 
     if (warp == 0) {
         if (lane == 0) {
@@ -576,7 +603,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool ok = true;
             const uint32_t tx_pair = 2u * (kABytes + boxes * kBBoxBytes);
             const uint32_t leader_full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
-            for (int t = pair; t < total_tiles && ok; t += npairs) {
+            for (int t = deal.first; t < total_tiles && ok; t += deal.stride) {
                 const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM, p.group_m);
                 const int my_row0 = ti.row0 + (int)rank * kBM;
                 const int wrow0 = ti.e * p.K;
@@ -585,7 +612,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         ok = false;  // test hook: both producers stop at the same stage
                         break;
                     }
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns) || s_abort) {
+                    if (!stage_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
                         record_error(p.err, kDeviceTimeoutBase | kRoleProducer);
                         ok = false;
                         break;
@@ -631,7 +658,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = pair; t < total_tiles && ok; t += npairs) {
+            for (int t = deal.first; t < total_tiles && ok; t += deal.stride) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns) || s_abort) {
                     record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                     ok = false;
@@ -640,7 +667,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * kAccCols;
                 for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!mbar_wait(&full_bar[stage], phase, p.timeout_ns) || s_abort) {
+                    if (!stage_wait(&full_bar[stage], phase, p.timeout_ns, s_abort)) {
                         record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                         ok = false;
                         break;
@@ -681,7 +708,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         const uint32_t leader_acc_empty0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
-        for (int t = pair; t < total_tiles; t += npairs) {
+        for (int t = deal.first; t < total_tiles; t += deal.stride) {
             const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM, p.group_m);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
