@@ -367,19 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&full_bar[stage], tx_bytes);
                     tma_load_2d(sA, &tmA, &full_bar[stage], kb * kBK, ti.row0);
                     const int wrow = wrow0 + kb * kBK;
+                    // Weight maps are 3-D views [chunk][row][64 columns] whose box
+                    // spans all the chunks of one copy: one load per matrix.
                     if (kSwiGLU) {
-                        // W1 columns [n0, n0 + half) then the same W3 columns
+                        // W1 columns [n0, n0 + half chunks) then the same W3 columns
                         const int half = p.n_boxes / 2;
-                        for (int j = 0; j < half; ++j) {
-                            tma_load_2d(sB + j * kBBoxBytes, &tmB0, &full_bar[stage],
-                                        ti.n0 + j * kBoxN, wrow);
-                            tma_load_2d(sB + (half + j) * kBBoxBytes, &tmB1, &full_bar[stage],
-                                        ti.n0 + j * kBoxN, wrow);
-                        }
+                        tma_load_3d(sB, &tmB0, &full_bar[stage], 0, wrow, ti.n0 / kBoxN);
+                        tma_load_3d(sB + half * kBBoxBytes, &tmB1, &full_bar[stage], 0, wrow,
+                                    ti.n0 / kBoxN);
                     } else {
-                        for (int j = 0; j < p.n_boxes; ++j)
-                            tma_load_2d(sB + j * kBBoxBytes, &tmB0, &full_bar[stage],
-                                        ti.n0 + j * kBoxN, wrow);
+                        tma_load_3d(sB, &tmB0, &full_bar[stage], 0, wrow, ti.n0 / kBoxN);
                     }
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -400,6 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             const uint32_t idesc = idesc_bf16_f32(kBM, p.n_boxes * kBoxN, false, true);
+            // Descriptors of stage 0, K step 0; a stage / K step only moves the
+            // start-address field (address >> 4, no carry below 256 KB).
+            const uint64_t adesc0 = desc_kmajor_sw128(smem_u32(smem));
+            const uint64_t bdesc0 = desc_mnmajor_sw128(smem_u32(smem) + kABytes, kBBoxBytes);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -420,14 +421,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
-                    const uint32_t b_addr = a_addr + kABytes;
+                    const uint64_t soff = (uint64_t)((uint32_t)(stage * kStageBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t adesc = desc_kmajor_sw128(a_addr + kk * 32);
-                        const uint64_t bdesc = desc_mnmajor_sw128(b_addr + kk * 2048, kBBoxBytes);
-                        tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0);
-                    }
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_bf16(d_tmem, adesc0 + soff + kk * (32 >> 4),
+                                    bdesc0 + soff + kk * (2048 >> 4), idesc, (kb | kk) != 0);
                     tc_commit(&empty_bar[stage]);
                     if (++stage == kStages) {
                         stage = 0;
@@ -625,12 +623,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const int wrow = wrow0 + kb * kBK;
                     if (kSwiGLU) {
                         const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
-                        tma_load_2d_pair(sB, mb, bar, ti.n0, wrow);
-                        tma_load_2d_pair(sB + kBBoxBytes, mb, bar, ti.n0 + kBoxN, wrow);
+                        tma_load_3d_pair(sB, mb, bar, 0, wrow, ti.n0 / kBoxN);
                     } else {
                         const int c0 = ti.n0 + (int)rank * boxes * kBoxN;
-                        for (int j = 0; j < boxes; ++j)
-                            tma_load_2d_pair(sB + j * kBBoxBytes, &tmB0, bar, c0 + j * kBoxN, wrow);
+                        tma_load_3d_pair(sB, &tmB0, bar, 0, wrow, c0 / kBoxN);
                     }
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -653,6 +649,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer (leader only)
             const uint32_t idesc = idesc_bf16_f32(kPM, 2 * boxes * kBoxN, false, true);
+            const uint64_t adesc0 = desc_kmajor_sw128(smem_u32(smem));
+            const uint64_t bdesc0 = desc_mnmajor_sw128(smem_u32(smem) + kABytes, kBBoxBytes);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -673,14 +671,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * kPairStageBytes);
-                    const uint32_t b_addr = a_addr + kABytes;
+                    const uint64_t soff = (uint64_t)((uint32_t)(stage * kPairStageBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t adesc = desc_kmajor_sw128(a_addr + kk * 32);
-                        const uint64_t bdesc = desc_mnmajor_sw128(b_addr + kk * 2048, kBBoxBytes);
-                        tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0);
-                    }
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_bf16_pair(d_tmem, adesc0 + soff + kk * (32 >> 4),
+                                         bdesc0 + soff + kk * (2048 >> 4), idesc, (kb | kk) != 0);
                     const uint32_t e_own = smem_u32(&empty_bar[stage]);
                     tc_commit_pair(e_own);
                     tc_commit_pair(map_to_cta(e_own, 1));
@@ -792,6 +787,25 @@ static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+// Weight map: a row-major [rows, cols] bf16 matrix viewed in 3-D as
+// [cols / 64 chunks][rows][64 columns] (chunk stride 128 bytes, row stride
+// cols * 2), box {64, 64 rows, chunks}, 128-byte swizzle.  One copy of the box
+// fills `chunks` consecutive 8 KB shared-memory boxes, each laid out exactly as
+// a 2-D {64, 64} box would be.
+static bool make_weight_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t chunks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)kBK, chunks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Output map for the epilogue's TMA stores: a row-major [rows, cols] matrix of
 // bf16 (h) or fp32 (o) with a 32 x 32-element box; the box rows are 64 or 128
 // bytes, swizzled in shared memory with the matching 64- or 128-byte pattern.
@@ -897,10 +911,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     if (!make_map(&mx, x_sorted, (uint64_t)R, (uint64_t)s.d, kBM) ||
         !make_map(&mh, h, (uint64_t)R, (uint64_t)s.d_ff, kBM) ||
         !make_out_map(&oh, h, (uint64_t)R, (uint64_t)s.d_ff, false) ||
-        !make_out_map(&oo, o, (uint64_t)R, (uint64_t)s.d, true) ||
-        !make_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
-        !make_map(&m3, W3, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, kBK) ||
-        !make_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, kBK))
+        !make_out_map(&oo, o, (uint64_t)R, (uint64_t)s.d, true))
         return MOE_ERR_CUDA;
     // GEMM2 (long K = d_ff) runs on CTA pairs (256-row tiles, M = 256 MMAs) once
     // there are at least kPairMinRows routed rows; GEMM1 (K = d, SwiGLU epilogue)
@@ -935,6 +946,12 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
     p1.bias_a = b1;
     p1.bias_b = b3;
+    // weight boxes: W1 / W3 chunks per copy = half of the CTA's B boxes (single
+    // CTA: both matrices) or all of them (pair: one matrix per CTA)
+    const uint32_t ch1 = pairs1 ? (uint32_t)p1.n_boxes : (uint32_t)p1.n_boxes / 2;
+    if (!make_weight_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1) ||
+        !make_weight_map(&m3, W3, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1))
+        return MOE_ERR_CUDA;
     const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / p1.n_tile_out);
     int rc = pairs1 ? launch_pair<true>(mx, m1, m3, oh, p1, t1, stream)
                     : launch<true>(mx, m1, m3, oh, p1, t1, stream);
@@ -952,6 +969,8 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.group_m = group_rows(pairs2 ? kPM : kBM, s.d_ff);
     p2.bias_a = b2;
     p2.bias_b = nullptr;
+    if (!make_weight_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, (uint32_t)p2.n_boxes))
+        return MOE_ERR_CUDA;
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
     return pairs2 ? launch_pair<false>(mh, m2, m2, oo, p2, t2, stream)
                   : launch<false>(mh, m2, m2, oo, p2, t2, stream);
