@@ -365,7 +365,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sA = smem + stage * kStageBytes;
                     uint8_t* sB = sA + kABytes;
                     mbar_arrive_expect_tx(&full_bar[stage], tx_bytes);
-                    tma_load_2d(sA, &tmA, &full_bar[stage], kb * kBK, ti.row0);
                     const int wrow = wrow0 + kb * kBK;
                     // Weight maps are 3-D views [chunk][row][64 columns] whose box
                     // spans all the chunks of one copy: one load per matrix.
@@ -378,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         tma_load_3d(sB, &tmB0, &full_bar[stage], 0, wrow, ti.n0 / kBoxN);
                     }
+                    tma_load_2d(sA, &tmA, &full_bar[stage], kb * kBK, ti.row0);
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     ++issued;
@@ -619,7 +619,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     uint8_t* sB = sA + kABytes;
                     const uint32_t bar = leader_full0 + stage * (uint32_t)sizeof(uint64_t);
                     if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx_pair);
-                    tma_load_2d_pair(sA, &tmA, bar, kb * kBK, my_row0);
                     const int wrow = wrow0 + kb * kBK;
                     if (kSwiGLU) {
                         const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
@@ -628,6 +627,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const int c0 = ti.n0 + (int)rank * boxes * kBoxN;
                         tma_load_3d_pair(sB, &tmB0, bar, 0, wrow, c0 / kBoxN);
                     }
+                    tma_load_2d_pair(sA, &tmA, bar, kb * kBK, my_row0);
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     ++issued;
