@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (rank 0) full barrier, which only the leader arms with the bytes of both;
 // the leader's single MMA thread commits each consumed stage to the empty
 // barriers of both CTAs and each finished accumulator to the acc_full barriers
-// of both; the epilogue warps of both CTAs arrive on the leader's acc_empty
+// of both (one multicast commit each); the epilogue warps of both CTAs arrive on the leader's acc_empty
 // barrier (count 8).  Cluster barriers at start (barrier initialisation) and
 // end (before the pair frees its tensor memory) are reached by every thread of
 // both CTAs unconditionally; every mbarrier wait in between is bounded.
@@ -676,18 +676,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < kBK / 16; ++kk)
                         tc_mma_bf16_pair(d_tmem, adesc0 + soff + kk * (32 >> 4),
                                          bdesc0 + soff + kk * (2048 >> 4), idesc, (kb | kk) != 0);
-                    const uint32_t e_own = smem_u32(&empty_bar[stage]);
-                    tc_commit_pair(e_own);
-                    tc_commit_pair(map_to_cta(e_own, 1));
+                    tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
                     if (++stage == kPairStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                const uint32_t f_own = smem_u32(&acc_full[acc]);
-                tc_commit_pair(f_own);
-                tc_commit_pair(map_to_cta(f_own, 1));
+                tc_commit_pair_mc(smem_u32(&acc_full[acc]), 0x3);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }

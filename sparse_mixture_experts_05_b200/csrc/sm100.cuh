@@ -89,16 +89,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map,
-                                                 uint64_t* bar, int32_t x, int32_t y,
-                                                 uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
-        : "memory");
-}
-
 // 3-D tiled load (x innermost); used for weight boxes of several adjacent
 // 64-column chunks in one copy.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
@@ -135,18 +125,6 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_group() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
 }
 
 // ------------------------------------------------------------------ tcgen05 / TMEM
@@ -300,6 +278,17 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             bar_cluster_addr)
+        : "memory");
+}
+
+// Arrives once on the mbarrier at the same shared-memory offset `bar_local` in
+// every CTA of `cta_mask` when every pair MMA issued so far has completed (one
+// commit for both CTAs of the pair).
+__device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar_local, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar_local),
+        "h"(cta_mask)
         : "memory");
 }
 
