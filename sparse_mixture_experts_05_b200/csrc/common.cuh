@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/moe.h"
 
@@ -58,6 +59,38 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // which measured slower at T = 4096.
 __device__ __forceinline__ void grid_dependency_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Raises `kernel`'s dynamic shared-memory limit to at least `bytes` on the
+// current device, calling the runtime only the first time (or when more is
+// needed): keeps the per-launch host path free of attribute calls, which also
+// keeps it legal inside stream capture.
+inline bool ensure_dynamic_smem(const void* kernel, int bytes) {
+    struct Entry {
+        const void* kernel;
+        int device;
+        int bytes;
+    };
+    static std::mutex mu;
+    static Entry cache[128];
+    static int n = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i) {
+        if (cache[i].kernel != kernel || cache[i].device != dev) continue;
+        if (cache[i].bytes >= bytes) return true;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess)
+            return false;
+        cache[i].bytes = bytes;
+        return true;
+    }
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return false;
+    if (n < 128) cache[n++] = Entry{kernel, dev, bytes};
+    return true;
 }
 
 // kernel<<<grid, block, smem, stream>>>(args...) with programmatic stream

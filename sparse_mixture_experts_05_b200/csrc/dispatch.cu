@@ -122,8 +122,7 @@ int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offse
                           cudaStream_t stream) {
     using namespace dispatch;
     const size_t smem = (size_t)s.E * kIndexThreads * sizeof(int);
-    if (cudaFuncSetAttribute(index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (!ensure_dynamic_smem(reinterpret_cast<const void*>(index_kernel), (int)smem))
         return MOE_ERR_CUDA;
     return launch_pdl(index_kernel, dim3(1), dim3(kIndexThreads), smem, stream, idx, s.T, s.E, s.k,
                       offsets, perm_tok, inv, status_to_clear) == cudaSuccess

@@ -664,23 +664,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * kAccCols;
+                // The next stage's barrier is looked at before this stage's MMAs
+                // are issued, so its wait overlaps them (measured faster here,
+                // not on the single-CTA kernel).
+                bool ready = mbar_try_wait(&full_bar[stage], phase);
                 for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!stage_wait(&full_bar[stage], phase, p.timeout_ns, s_abort)) {
+                    if (!ready && !stage_wait(&full_bar[stage], phase, p.timeout_ns, s_abort)) {
                         record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                         ok = false;
                         break;
                     }
-                    tc_fence_after_sync();
-                    const uint64_t soff = (uint64_t)((uint32_t)(stage * kPairStageBytes) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma_bf16_pair(d_tmem, adesc0 + soff + kk * (32 >> 4),
-                                         bdesc0 + soff + kk * (2048 >> 4), idesc, (kb | kk) != 0);
-                    tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
+                    const int cur = stage;
                     if (++stage == kPairStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
+                    ready = kb + 1 < kb_count && mbar_try_wait(&full_bar[stage], phase);
+                    const uint64_t soff = (uint64_t)((uint32_t)(cur * kPairStageBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_bf16_pair(d_tmem, adesc0 + soff + kk * (32 >> 4),
+                                         bdesc0 + soff + kk * (2048 >> 4), idesc, (kb | kk) != 0);
+                    tc_commit_pair_mc(smem_u32(&empty_bar[cur]), 0x3);
                 }
                 if (!ok) break;
                 tc_commit_pair_mc(smem_u32(&acc_full[acc]), 0x3);

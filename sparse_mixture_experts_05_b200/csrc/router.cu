@@ -245,8 +245,7 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
     const uint16_t* xp = static_cast<const uint16_t*>(x);
     const uint16_t* wp = static_cast<const uint16_t*>(Wg);
     auto run = [&](auto kern) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
+        if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem))
             return MOE_ERR_CUDA;
         return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, xp, wp, bias, s.T, s.d,
                           s.E, s.k, idx, gate, logits) == cudaSuccess
