@@ -18,7 +18,11 @@ namespace moe {
 namespace combine {
 
 // One thread per (token, 8-column chunk): at small T this spreads the few rows
-// over the whole GPU instead of one warp per row.
+// over the whole GPU instead of one warp per row.  All of a thread's inverse-map
+// and gate loads are issued first, then all of its expert-row loads, so the
+// row loads do not wait on each other.  KMAX >= k bounds the slot arrays (2 for
+// the common top-2, 8 otherwise).
+template <int KMAX>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ inv,
                    const float* __restrict__ gate, int T, int d8, int k,
@@ -29,20 +33,33 @@ __global__ void __launch_bounds__(256)
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
         const int t = (int)(i / d8);
         const int c = (int)(i - (int64_t)t * d8);
+        int rows[KMAX];
+        float gs[KMAX];
+#pragma unroll
+        for (int s = 0; s < KMAX; ++s) {
+            rows[s] = s < k ? __ldg(inv + (int64_t)t * k + s) : -1;
+            gs[s] = s < k ? __ldg(gate + (int64_t)t * k + s) : 0.f;
+        }
+        float4 v[KMAX][2];
+#pragma unroll
+        for (int s = 0; s < KMAX; ++s) {
+            // a skipped slot (row < 0) reads row 0, which always exists, and is ignored
+            const float4* src = o + ((int64_t)(rows[s] < 0 ? 0 : rows[s]) * d8 + c) * 2;
+            if (s < k) {
+                v[s][0] = __ldg(src);
+                v[s][1] = __ldg(src + 1);
+            }
+        }
         float acc[8];
         bool first = true;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            if (s >= k) break;
-            const int row = __ldg(inv + (int64_t)t * k + s);
-            if (row < 0) continue;
-            const float g = __ldg(gate + (int64_t)t * k + s);
-            const float4* src = o + ((int64_t)row * d8 + c) * 2;
-            const float4 v0 = __ldg(src);
-            const float4 v1 = __ldg(src + 1);
-            const float p[8] = {__fmul_rn(g, v0.x), __fmul_rn(g, v0.y), __fmul_rn(g, v0.z),
-                                __fmul_rn(g, v0.w), __fmul_rn(g, v1.x), __fmul_rn(g, v1.y),
-                                __fmul_rn(g, v1.z), __fmul_rn(g, v1.w)};
+        for (int s = 0; s < KMAX; ++s) {
+            if (s >= k || rows[s] < 0) continue;
+            const float g = gs[s];
+            const float p[8] = {__fmul_rn(g, v[s][0].x), __fmul_rn(g, v[s][0].y),
+                                __fmul_rn(g, v[s][0].z), __fmul_rn(g, v[s][0].w),
+                                __fmul_rn(g, v[s][1].x), __fmul_rn(g, v[s][1].y),
+                                __fmul_rn(g, v[s][1].z), __fmul_rn(g, v[s][1].w)};
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = first ? p[j] : __fadd_rn(acc[j], p[j]);
             first = false;
@@ -74,9 +91,10 @@ int launch_combine(const moe_shape& s, const float* o, const int32_t* inv, const
     const int64_t work = (int64_t)s.T * (s.d / 8);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256,
                                                                  (int64_t)device_sm_count() * 8));
-    return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, stream,
-                      reinterpret_cast<const float4*>(o), inv, gate, s.T, s.d / 8, s.k,
-                      static_cast<const uint4*>(residual), static_cast<uint4*>(y)) == cudaSuccess
+    auto kern = s.k <= 2 ? combine_kernel<2> : combine_kernel<8>;
+    return launch_pdl(kern, dim3(grid), dim3(256), 0, stream, reinterpret_cast<const float4*>(o),
+                      inv, gate, s.T, s.d / 8, s.k, static_cast<const uint4*>(residual),
+                      static_cast<uint4*>(y)) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

@@ -7,10 +7,11 @@
 // an exclusive scan of the per-expert counts produces.
 //
 // Two launches:
-//  1. index kernel (one CTA of 1024 threads): thread i owns a contiguous run of
-//     tokens; per-thread per-expert counts, an exclusive scan over threads for
-//     each expert, then each thread walks its run again and hands out positions
-//     in token order.  Integer-only and deterministic (no atomics on positions).
+//  1. index kernel (one CTA of 1024 threads): each warp owns a contiguous run
+//     of slots; warp-wide grouping by expert id (__match_any_sync) gives counts
+//     and in-order ranks, one warp scans the per-warp counts into offsets and
+//     starting positions, and a second pass hands out positions in token order.
+//     Integer-only and deterministic (no atomics on positions).
 //  2. scatter kernel: reads each x row once and writes it to its k sorted rows
 //     (16-byte vector copies, one thread per 16-byte chunk).
 #include <cuda_runtime.h>
@@ -23,74 +24,92 @@
 namespace moe {
 namespace dispatch {
 
-constexpr int kIndexThreads = 1024;
+constexpr int kIndexThreads = 1024;  // 32 warps
+constexpr int kIndexWarps = kIndexThreads / 32;
+constexpr int kMaxExperts = 32;
 
-__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, v, off);
-        if (lane >= off) v += o;
-    }
-    return v;
-}
-
+// One CTA.  The T*k slots (slot j = t*k + s, ascending in t) are cut into 32
+// contiguous runs, one per warp, taken 32 slots at a time.  In each group of
+// 32 slots, __match_any_sync on the expert id gives every lane the lanes that
+// chose the same expert: their number and this lane's rank among them (lane
+// order = slot order).  Pass 1 sums the per-warp, per-expert counts; one warp
+// turns them into offsets and per-warp starting positions (expert-major, then
+// warp order); pass 2 repeats the grouping and hands out positions.  Stable
+// (slot order within each expert), deterministic, no atomics.
 __global__ void __launch_bounds__(kIndexThreads, 1)
     index_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                  int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
                  int32_t* __restrict__ inv, int* status_to_clear) {
-    extern __shared__ int s_cnt[];  // [E][1024]: entries of expert e in thread i's run
-    __shared__ int s_total[32];
-    __shared__ int s_base[33];
+    __shared__ int s_pos[kIndexWarps][kMaxExperts + 1];  // counts, then next positions
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     grid_dependency_wait();
     if (status_to_clear && tid == 0) *status_to_clear = 0;
 
-    const int per = (T + kIndexThreads - 1) / kIndexThreads;
-    const int t_begin = min(T, tid * per);
-    const int t_end = min(T, t_begin + per);
+    const int n = T * k;
+    const int per_warp = ((n + kIndexWarps - 1) / kIndexWarps + 31) / 32 * 32;
+    const int j0 = min(n, warp * per_warp);
+    const int j1 = min(n, j0 + per_warp);
+    const unsigned lt_mask = (1u << lane) - 1u;
 
-    for (int e = 0; e < E; ++e) s_cnt[e * kIndexThreads + tid] = 0;
-    for (int t = t_begin; t < t_end; ++t)
-        for (int s = 0; s < k; ++s) {
-            const int e = idx[(int64_t)t * k + s];
-            if (e >= 0 && e < E) s_cnt[e * kIndexThreads + tid] += 1;
-        }
-    __syncthreads();
-
-    // Exclusive scan over threads (= over token runs in order), one warp per expert.
-    if (warp < E) {
-        int carry = 0;
-        for (int c = 0; c < kIndexThreads; c += 32) {
-            const int v = s_cnt[warp * kIndexThreads + c + lane];
-            const int incl = warp_inclusive_scan(v, lane);
-            s_cnt[warp * kIndexThreads + c + lane] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) s_total[warp] = carry;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        s_base[0] = 0;
-        for (int e = 0; e < E; ++e) s_base[e + 1] = s_base[e] + s_total[e];
-        for (int e = 0; e <= E; ++e) offsets[e] = s_base[e];
+    if (lane <= kMaxExperts) s_pos[warp][lane] = 0;
+    __syncwarp();
+    // pass 1: per-warp counts
+    for (int base = j0; base < j1; base += 32) {
+        const int j = base + lane;
+        const int e = j < j1 ? idx[j] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
+        if (valid && (same & lt_mask) == 0) s_pos[warp][e] += __popc(same);
+        __syncwarp();
     }
     __syncthreads();
 
-    for (int e = 0; e < E; ++e) s_cnt[e * kIndexThreads + tid] += s_base[e];
-    for (int t = t_begin; t < t_end; ++t)
-        for (int s = 0; s < k; ++s) {
-            const int64_t j = (int64_t)t * k + s;
-            const int e = idx[j];
-            if (e >= 0 && e < E) {
-                const int pos = s_cnt[e * kIndexThreads + tid]++;
-                perm_tok[pos] = t;
-                inv[j] = pos;
-            } else {
-                inv[j] = -1;
+    // offsets and per-warp starting positions (warp 0, lane = expert)
+    if (warp == 0) {
+        int total = 0;
+        if (lane < E)
+            for (int w = 0; w < kIndexWarps; ++w) {
+                const int c = s_pos[w][lane];
+                s_pos[w][lane] = total;  // position of this warp's first row of expert `lane`, relative
+                total += c;
             }
+        // exclusive scan of the totals over experts
+        int incl = total;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
         }
+        const int excl = incl - total;
+        if (lane < E) {
+            offsets[lane] = excl;
+            for (int w = 0; w < kIndexWarps; ++w) s_pos[w][lane] += excl;
+        }
+        const int all = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0) offsets[E] = all;
+    }
+    __syncthreads();
+
+    // pass 2: positions in slot order
+    for (int base = j0; base < j1; base += 32) {
+        const int j = base + lane;
+        const bool in = j < j1;
+        const int e = in ? idx[j] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
+        if (valid) {
+            const int pos = s_pos[warp][e] + __popc(same & lt_mask);
+            perm_tok[pos] = j / k;
+            inv[j] = pos;
+        } else if (in) {
+            inv[j] = -1;
+        }
+        __syncwarp();
+        if (valid && (same & lt_mask) == 0) s_pos[warp][e] += __popc(same);
+        __syncwarp();
+    }
 }
 
 // x_sorted[inv[t, s]] = x[t] for every slot s of token t; one thread per
@@ -121,10 +140,8 @@ int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offse
                           int32_t* perm_tok, int32_t* inv, int* status_to_clear,
                           cudaStream_t stream) {
     using namespace dispatch;
-    const size_t smem = (size_t)s.E * kIndexThreads * sizeof(int);
-    if (!ensure_dynamic_smem(reinterpret_cast<const void*>(index_kernel), (int)smem))
-        return MOE_ERR_CUDA;
-    return launch_pdl(index_kernel, dim3(1), dim3(kIndexThreads), smem, stream, idx, s.T, s.E, s.k,
+    if (s.E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    return launch_pdl(index_kernel, dim3(1), dim3(kIndexThreads), 0, stream, idx, s.T, s.E, s.k,
                       offsets, perm_tok, inv, status_to_clear) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
