@@ -1,5 +1,6 @@
 """Mixtral 8x7B shapes at full size (d = 4096, d_ff = 14336, E = 8, k = 2):
-prefill T = 4096, decode T = 16, skewed prefill T = 16384 with router bias.
+prefill T = 4096, decode T = 16, skewed prefill T = 16384 with router bias, and
+a T = 65536 batch near the largest the library accepts.
 
 Routing is checked on every token; the expert kernel on sampled sorted rows
 (including the last row of every expert group, where tiles are ragged); the
@@ -19,9 +20,12 @@ from _parity import bf16_values, check_expert_rows, check_routing, check_y, to_d
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module", params=["decode", "prefill", "skew"])
+@pytest.fixture(scope="module", params=["decode", "prefill", "skew", "max"])
 def case(request):
-    inp = workload_inputs(request.param)
+    # "max": the prefill recipe at T = 65536, close to the largest batch the
+    # library accepts at these widths (T * k * d_ff < 2^31)
+    inp = (workload_inputs("prefill", T=65536) if request.param == "max"
+           else workload_inputs(request.param))
     dev = to_dev(inp)
     T, d, d_ff, E, k = inp["shape"]
     idx = torch.empty(T, k, dtype=torch.int32, device="cuda")

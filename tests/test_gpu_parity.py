@@ -27,6 +27,7 @@ CASES = {
     "E1k1": (40, 128, 128, 1, 1, 8, False),
     "E16k4": (96, 256, 256, 16, 4, 9, False),
     "E5k3": (33, 128, 256, 5, 3, 10, False),
+    "E32k8": (64, 128, 256, 32, 8, 18, False),    # the largest E and k the library takes
     "single": (1, 128, 256, 8, 2, 11, False),
     "batch16": (16, 256, 384, 8, 2, 16, True),    # decode-sized: R = 32 rows over 8 experts
     "batch30": (30, 128, 512, 8, 2, 17, False),
