@@ -214,9 +214,14 @@ int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, 
 
 /*
  * moe_forward_hostio -- moe_forward with x and y in HOST memory (pinned memory
- * gives asynchronous copies): enqueues the host->device copy of x into the
- * workspace, the layer, and the device->host copy of y, all on `stream`.  The
- * caller synchronises the stream before reading y.  Weights stay on the device.
+ * gives asynchronous copies): copies x into the workspace, runs the layer and
+ * copies y back; everything is ordered after earlier work on `stream`, and
+ * `stream` is ordered after the last copy, so the caller synchronises `stream`
+ * before reading y.  Weights stay on the device.  Batches of 2048 tokens or
+ * more are split into two token halves whose copies run on two library-owned
+ * copy streams (created once per device) while the other half computes:
+ * the layer is independent per token, so y is the same bit for bit.  Calls
+ * from several host threads on one device are enqueued one at a time.
  *   ws: >= moe_forward_workspace_bytes(s) + T*d*2 (x staging) + T*d*2 (y staging)
  *       bytes; moe_forward_hostio_workspace_bytes gives the exact figure.
  */

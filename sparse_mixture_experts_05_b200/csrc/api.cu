@@ -100,7 +100,8 @@ struct ExpertBias {
 int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                  const void* W1, const void* W3, const void* W2, void* y, int32_t* idx_out,
                  float* gate_out, void* ws, cudaStream_t st, void* const* events,
-                 const void* residual = nullptr, const ExpertBias& eb = ExpertBias{}) {
+                 const void* residual = nullptr, const ExpertBias& eb = ExpertBias{},
+                 int router_split = 0) {
     auto mark = [&](int i) {
         return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
     };
@@ -115,7 +116,7 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     float* o = at<float>(ws, L.o);
     int* status = at<int>(ws, L.hdr);
     if (!mark(0)) return MOE_ERR_CUDA;
-    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st);
+    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, router_split);
     if (rc) return rc;
     if (!mark(1)) return MOE_ERR_CUDA;
     rc = launch_dispatch_index(s, idx, offsets, perm, inv, status, st);
@@ -154,6 +155,39 @@ void* static_scratch_address() {
         addr[dev] = p;
     }
     return addr[dev];
+}
+
+// moe_forward_hostio splits batches of 2048+ tokens into two halves whose copies
+// overlap the other half's computation.  (Four chunks measured slower: at 1024
+// tokens the down projection's CTA-pair tiles fill only 2.2 of 3 rounds.)
+constexpr int kMaxHostioChunks = 2;
+int hostio_chunks(int T) { return T >= 2048 ? 2 : 1; }
+
+// Two copy streams (host->device, device->host) and the events that order them
+// against the caller's stream; created once per device and kept for the life
+// of the process.  The mutex serialises the enqueueing of one call's pipeline.
+struct CopyStreams {
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t ev[2 + 2 * kMaxHostioChunks] = {};
+    std::mutex mu;
+};
+
+CopyStreams* copy_streams() {
+    static std::mutex mu;
+    static CopyStreams* per_device[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!per_device[dev]) {
+        CopyStreams* cs = new CopyStreams();
+        bool ok = cudaStreamCreateWithFlags(&cs->up, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&cs->down, cudaStreamNonBlocking) == cudaSuccess;
+        for (auto& e : cs->ev)
+            ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return nullptr;  // (leaks the partial set; only on a failing device)
+        per_device[dev] = cs;
+    }
+    return per_device[dev];
 }
 
 }  // namespace
@@ -353,15 +387,57 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t fwd = moe_forward_workspace_bytes(s);
     const size_t io_bytes = (size_t)s.T * s.d * 2;
-    void* x_dev = static_cast<char*>(ws) + fwd;
-    void* y_dev = static_cast<char*>(ws) + fwd + align_up(io_bytes, 256);
-    if (cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    rc = forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st, nullptr);
-    if (rc) return rc;
-    if (cudaMemcpyAsync(y_host, y_dev, io_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    return MOE_OK;
+    char* x_dev = static_cast<char*>(ws) + fwd;
+    char* y_dev = static_cast<char*>(ws) + fwd + align_up(io_bytes, 256);
+    const int chunks = hostio_chunks(s.T);
+    if (chunks == 1) {
+        if (cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        rc = forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st,
+                          nullptr);
+        if (rc) return rc;
+        if (cudaMemcpyAsync(y_host, y_dev, io_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    // Token chunks in a pipeline: the layer is independent per token, so chunk c
+    // computes (on `st`) while chunk c+1's x is still arriving and chunk c-1's y
+    // is leaving, on the two copy engines.  The result equals the unchunked
+    // layer bit for bit: no row's arithmetic depends on the other rows.
+    CopyStreams* cs = copy_streams();
+    if (!cs) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(cs->mu);
+    const int per = (s.T + chunks - 1) / chunks;
+    const int split = router_ksplit(s);  // the whole batch's: every chunk rounds alike
+    const size_t row_bytes = (size_t)s.d * 2;
+    bool ok = cudaEventRecord(cs->ev[0], st) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->up, cs->ev[0], 0) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->down, cs->ev[0], 0) == cudaSuccess;
+    for (int c = 0; ok && c < chunks; ++c) {
+        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
+        ok = cudaMemcpyAsync(x_dev + t0 * row_bytes, static_cast<const char*>(x_host) + t0 * row_bytes,
+                             (size_t)tn * row_bytes, cudaMemcpyHostToDevice, cs->up) == cudaSuccess &&
+             cudaEventRecord(cs->ev[1 + c], cs->up) == cudaSuccess;
+    }
+    for (int c = 0; ok && c < chunks; ++c) {
+        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
+        moe_shape sc = s;
+        sc.T = tn;
+        ok = cudaStreamWaitEvent(st, cs->ev[1 + c], 0) == cudaSuccess &&
+             forward_impl(sc, x_dev + t0 * row_bytes, Wg, bias, W1, W3, W2, y_dev + t0 * row_bytes,
+                          nullptr, nullptr, ws, st, nullptr, nullptr, ExpertBias{},
+                          split) == MOE_OK &&
+             cudaEventRecord(cs->ev[1 + kMaxHostioChunks + c], st) == cudaSuccess &&
+             cudaStreamWaitEvent(cs->down, cs->ev[1 + kMaxHostioChunks + c], 0) == cudaSuccess &&
+             cudaMemcpyAsync(static_cast<char*>(y_host) + t0 * row_bytes, y_dev + t0 * row_bytes,
+                             (size_t)tn * row_bytes, cudaMemcpyDeviceToHost,
+                             cs->down) == cudaSuccess;
+    }
+    // join: the caller's stream waits for the last copy back
+    const int last = 1 + 2 * kMaxHostioChunks;
+    ok = ok && cudaEventRecord(cs->ev[last], cs->down) == cudaSuccess &&
+         cudaStreamWaitEvent(st, cs->ev[last], 0) == cudaSuccess;
+    return ok ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int moe_forward_static(moe_shape s, const void* x, const void* Wg, const float* bias,

@@ -221,25 +221,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace router
 
+int router_ksplit(const moe_shape& s) {
+    using namespace router;
+    const int ntiles = (s.T + 15) / 16;
+    const int sms = device_sm_count();
+    // Largest split of d (into 16, 8 or 4 parts, each a whole number of 32-wide
+    // k blocks) that still needs no more CTAs than there are SMs: few tokens
+    // (decode) then get 16 warps per tile instead of 4.
+    for (int cand : {16, 8}) {
+        const int ctas = (ntiles * cand + kWarps - 1) / kWarps;
+        if ((s.d / 32) % cand == 0 && ctas <= sms) return cand;
+    }
+    return 4;
+}
+
 int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
-                  int32_t* idx, float* gate, float* logits, cudaStream_t stream) {
+                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int ksplit) {
     using namespace router;
     if (s.T == 0) return MOE_OK;
     const int NT = (s.E + 7) / 8;
     const size_t smem = (size_t)s.d * NT * 16;
     const int ntiles = (s.T + 15) / 16;
     const int sms = device_sm_count();
-    // Largest split of d (into 16, 8 or 4 parts, each a whole number of 32-wide
-    // k blocks) that still needs no more CTAs than there are SMs: few tokens
-    // (decode) then get 16 warps per tile instead of 4.
-    int ksplit = 4;
-    for (int cand : {16, 8}) {
-        const int ctas = (ntiles * cand + kWarps - 1) / kWarps;
-        if ((s.d / 32) % cand == 0 && ctas <= sms) {
-            ksplit = cand;
-            break;
-        }
-    }
+    // The split decides the order in which the partial sums of a logit are
+    // added; a caller that runs one batch in token chunks passes the split of
+    // the whole batch so every chunk rounds the same way.
+    if (ksplit <= 0) ksplit = router_ksplit(s);
+    if (ksplit != 4 && ksplit != 8 && ksplit != 16) return MOE_ERR_INVALID_ARG;
+    if ((s.d / 32) % ksplit != 0) return MOE_ERR_INVALID_ARG;
     const int slots = kWarps / ksplit;
     const int grid = std::max(1, std::min(sms, (ntiles + slots - 1) / slots));
     const uint16_t* xp = static_cast<const uint16_t*>(x);
