@@ -15,12 +15,18 @@
 // K advances 64 elements (one 128-byte swizzle row) per pipeline stage.
 //
 // Roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: A box [128 x 64] (K-major) + B boxes [64 x 64] (MN-major)
+//   warp 0      TMA producer: per stage one copy per weight matrix (a 3-D box
+//               filling 64 x 64 MN-major boxes, see make_weight_map), issued
+//               first, then the A box [128 x 64] (K-major)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 2..5  epilogue: tcgen05.ld -> SiLU(.) / convert -> TMA stores of 32 x 32 chunks
 // Shared-memory stages are recycled through full/empty mbarriers; the two TMEM
 // accumulator buffers (2 x 256 columns) let the epilogue of tile i overlap the
-// MMAs of tile i+1.
+// MMAs of tile i+1.  The producer and MMA stage loops are on the critical path
+// (every stage waits for a load round trip), so they are kept short: the abort
+// flag is read only after a slow wait, descriptors are derived by addition.
+// Tiles are dealt evenly to the CTAs (deal_tiles); the CTA-pair variant for the
+// down projection is described further below.
 //
 // Weights stay in their natural row-major layout ([E, d, d_ff] and
 // [E, d_ff, d]); the B operand is read MN-major, which tcgen05 supports for
