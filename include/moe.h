@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, k outside 1..E, negative size */
-    MOE_ERR_UNSUPPORTED = 2,    /* legal shape this build does not handle (see limits above) */
+    MOE_ERR_UNSUPPORTED = 2,    /* legal shape the library does not handle (see limits above) */
     MOE_ERR_WORKSPACE = 3,      /* workspace smaller than the matching *_workspace_bytes */
     MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
     MOE_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait expired (see moe_read_device_status) */
