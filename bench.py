@@ -312,6 +312,52 @@ def timed_loop(ctx, steps, pg, device, clock, profiled):
     return step_ms, parts, outer0.elapsed_time(outer1), clocks
 
 
+def extras_loop(ctx, steps, device):
+    """The widened entry points on the same batch (each timed like the plain step,
+    L2 flushed before each call): the block with its edges, the layer with expert
+    biases, and the load-balancing term on the router's logits."""
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    from sparse_mixture_experts_05_b200.inputs import expert_biases
+    inp = ctx["inp"]
+    shape = ctx["shape"]
+    T, d, d_ff, E, k = shape
+    x, Wg, bias, W1, W3, W2 = (inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(5)
+    gamma = (1 + 0.2 * torch.randn(d, generator=gen, device=device)).to(torch.bfloat16)
+    eb = expert_biases(E, d, d_ff, seed=6, device=device)
+    ws_b = moe.workspace(moe.moe_block_workspace_bytes(shape), device)
+    H = torch.empty(T, d, dtype=torch.bfloat16, device=device)
+    idx, _, logits = moe.moe_route(shape, x, Wg, bias, want_logits=True)
+    calls = {
+        "block_forward_ms": lambda: moe.moe_block_forward(shape, x, gamma, Wg, bias, W1, W3, W2,
+                                                          H=H, ws=ws_b),
+        "forward_bias_ms": lambda: moe.moe_forward_bias(shape, x, Wg, bias, W1, W3, W2, eb,
+                                                        y=ctx["y"], ws=ctx["ws"]),
+        "aux_loss_ms": lambda: moe.moe_aux_loss(shape, logits, idx),
+    }
+    out = {}
+    for name, call in calls.items():
+        for _ in range(3):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for i in range(steps):
+            ctx["flush"].fill_(i & 0xFF)
+            evs[i][0].record()
+            call()
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        out[name] = round(statistics.mean(a.elapsed_time(b) for a, b in evs), 4)
+    if moe.moe_read_device_status(ws_b) != moe.MOE_OK:
+        raise RuntimeError("device status error in the block forward")
+    out["note"] = ("same batch; block = RMSNorm + layer + residual; bias = expert Linear "
+                   "biases b1, b3, b2; aux = load-balancing term over the T x E logits")
+    return out
+
+
 def e2e_loop(ctx, steps, warmup, device):
     import torch
 
@@ -445,6 +491,8 @@ def run_ours(a):
         "tflops_layer": round(alg["flops_total"] / (max_ms / 1000) / 1e12, 1),
         "bracket_ms_incl_flush": round(bracket_ms, 3),
     }
+    if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
+        line["extras"] = extras_loop(ctx, a.steps, device)
     del ctx
     torch.cuda.empty_cache()
 
