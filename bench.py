@@ -497,18 +497,20 @@ def run_ours(a):
     torch.cuda.empty_cache()
 
     if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
-        dctx = time_workload("decode", a.steps, a.warmup, device, rank)
-        d_ms, _, _, d_clocks = timed_loop(dctx, a.steps, pg, device, ClockSampler(local),
+        # a decode step is ~0.5 ms: time at least 40 of them so the mean is stable
+        d_steps = max(a.steps, 40)
+        dctx = time_workload("decode", d_steps, a.warmup, device, rank)
+        d_ms, _, _, d_clocks = timed_loop(dctx, d_steps, pg, device, ClockSampler(local),
                                           profiled=False)
         d_mean = reduce_max(pg, statistics.mean(d_ms), device)
-        d_pms, d_parts, _, _ = timed_loop(dctx, a.steps, pg, device, None, profiled=True)
+        d_pms, d_parts, _, _ = timed_loop(dctx, d_steps, pg, device, None, profiled=True)
         d_pmean = reduce_max(pg, statistics.mean(d_pms), device)
         d_alg = algorithmic(dctx["shape"], dctx["counts"])
         d_gemm = d_parts["gemm1_swiglu"] + d_parts["gemm2_down"]
         d_gbs = d_alg["bytes_experts_decode"] / (d_gemm / 1000) / 1e9
         line["decode"] = {
             "workload": WORKLOAD_NAMES["decode"], "tokens_per_s": round(16 * world / (d_mean / 1e3), 1),
-            "ms_per_step": round(d_mean, 4),
+            "ms_per_step": round(d_mean, 4), "steps": d_steps,
             "experts_gbs": round(d_gbs, 1), "frac_of_measured_hbm": round(d_gbs / peaks["hbm_gbs"], 4),
             "frac_of_spec_8000": round(d_gbs / SPEC_HBM_GBS, 4),
             "layer_gbs": round((d_alg["bytes_experts_decode"] + d_alg["bytes_router"]) /

@@ -27,6 +27,7 @@ namespace dispatch {
 constexpr int kIndexThreads = 1024;  // 32 warps
 constexpr int kIndexWarps = kIndexThreads / 32;
 constexpr int kMaxExperts = 32;
+constexpr int kBatch = 8;  // groups of 32 slots whose ids are loaded together
 
 // One CTA.  The T*k slots (slot j = t*k + s, ascending in t) are cut into 32
 // contiguous runs, one per warp, taken 32 slots at a time.  In each group of
@@ -55,14 +56,23 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
 
     if (lane <= kMaxExperts) s_pos[warp][lane] = 0;
     __syncwarp();
-    // pass 1: per-warp counts
-    for (int base = j0; base < j1; base += 32) {
-        const int j = base + lane;
-        const int e = j < j1 ? idx[j] : -1;
-        const bool valid = e >= 0 && e < E;
-        const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
-        if (valid && (same & lt_mask) == 0) s_pos[warp][e] += __popc(same);
-        __syncwarp();
+    // pass 1: per-warp counts (the ids of kBatch groups are loaded before any is
+    // used, so their load latencies overlap)
+    for (int base = j0; base < j1; base += 32 * kBatch) {
+        int ids[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = base + u * 32 + lane;
+            ids[u] = j < j1 ? idx[j] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = ids[u];
+            const bool valid = e >= 0 && e < E;
+            const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
+            if (valid && (same & lt_mask) == 0) s_pos[warp][e] += __popc(same);
+            __syncwarp();
+        }
     }
     __syncthreads();
 
@@ -93,22 +103,31 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
     __syncthreads();
 
     // pass 2: positions in slot order
-    for (int base = j0; base < j1; base += 32) {
-        const int j = base + lane;
-        const bool in = j < j1;
-        const int e = in ? idx[j] : -1;
-        const bool valid = e >= 0 && e < E;
-        const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
-        if (valid) {
-            const int pos = s_pos[warp][e] + __popc(same & lt_mask);
-            perm_tok[pos] = j / k;
-            inv[j] = pos;
-        } else if (in) {
-            inv[j] = -1;
+    for (int base = j0; base < j1; base += 32 * kBatch) {
+        int ids[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = base + u * 32 + lane;
+            ids[u] = j < j1 ? idx[j] : -1;
         }
-        __syncwarp();
-        if (valid && (same & lt_mask) == 0) s_pos[warp][e] += __popc(same);
-        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = base + u * 32 + lane;
+            const bool in = j < j1;
+            const int e = ids[u];
+            const bool valid = e >= 0 && e < E;
+            const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
+            if (valid) {
+                const int pos = s_pos[warp][e] + __popc(same & lt_mask);
+                perm_tok[pos] = j / k;
+                inv[j] = pos;
+            } else if (in) {
+                inv[j] = -1;
+            }
+            __syncwarp();
+            if (valid && (same & lt_mask) == 0) s_pos[warp][e] += __popc(same);
+            __syncwarp();
+        }
     }
 }
 

@@ -58,6 +58,21 @@ def test_route(name):
     check_routing(idx.cpu().numpy(), gate.cpu().numpy(), o_idx, o_gate, o_logits, k)
 
 
+@pytest.mark.parametrize("T,d,E,k", [(40, 10240, 8, 2), (40, 8192, 8, 2), (40, 2560, 32, 8)],
+                         ids=["d10240", "d8192", "E32-d2560"])
+def test_route_wide_rows(T, d, E, k):
+    # W_r staged in shared memory near the largest size the library takes (160 KB)
+    inp = make_inputs(T, d, 128, E, k, seed=20 + E, bias=True)
+    dev = to_dev(inp)
+    idx, gate, logits = moe.moe_route(inp["shape"], dev["x"], dev["Wg"], dev["bias"],
+                                      want_logits=True)
+    torch.cuda.synchronize()
+    o_idx, o_gate, o_logits = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    lerr = np.max(np.abs(logits.cpu().numpy() - o_logits))
+    assert lerr < 1e-4, lerr
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), o_idx, o_gate, o_logits, k)
+
+
 def test_route_ties_to_lower_index():
     inp = make_inputs(48, 128, 256, 8, 2, seed=12)
     inp["Wg"][:, 6] = inp["Wg"][:, 3]
