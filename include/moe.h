@@ -117,7 +117,9 @@ int moe_dispatch(moe_shape s, const int32_t* idx, const void* x, int32_t* offset
  *   o [T*k,d] float:   h W2_e (out)
  *   ws: >= moe_expert_workspace_bytes(s) bytes of device memory (scratch)
  * Rows at or beyond offsets[E] are left untouched; an expert without rows
- * costs nothing.  A device wait that expires leaves o/h incomplete and is
+ * costs nothing.  Each row's h and o are accumulated in one fixed order
+ * whatever the other rows are, so running an expert's rows alone gives the
+ * same bits.  A device wait that expires leaves o/h incomplete and is
  * reported by moe_read_device_status(ws).
  */
 int moe_expert_swiglu(moe_shape s, const void* x_sorted, const int32_t* offsets, const void* W1,

@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 int launch_aux_loss(const moe_shape& s, const float* logits, const int32_t* idx,
                     const uint8_t* mask, float* aux_out, float* f_out, float* P_out,
                     cudaStream_t stream) {
+    if (s.E > aux::kMaxE || s.k > aux::kMaxK) return MOE_ERR_UNSUPPORTED;
     auto kern = s.E <= 8 ? aux::aux_loss_kernel<8>
                 : (s.E <= 16 ? aux::aux_loss_kernel<16> : aux::aux_loss_kernel<32>);
     kern<<<1, aux::kThreads, 0, stream>>>(logits, idx, mask, s.T, s.E, s.k, aux_out, f_out, P_out);
