@@ -64,6 +64,9 @@ def parse(argv=None):
                     help="override T (smaller cases for profiler captures)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (smaller cases for profiler captures)")
+    ap.add_argument("--vs-cublas", action="store_true",
+                    help="instead of the step: time the expert GEMMs against cuBLAS batched "
+                         "bf16 GEMMs of the same shapes (equal rows per expert), alternating")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -587,10 +590,87 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+def vs_cublas(a):
+    """The expert GEMMs (one moe_expert_swiglu call: GEMM1 with the SwiGLU epilogue,
+    then GEMM2) against cuBLAS batched bf16 GEMMs of the same shapes through torch
+    (x [E, R/E, d] . [W1|W3] [E, d, 2 d_ff], then h [E, R/E, d_ff] . W2 [E, d_ff, d]),
+    with R/E rows per expert so neither side pads.  The two alternate step by step
+    with the L2 flushed before each, so both see the same clocks and power state.
+    cuBLAS writes bf16 outputs and has no SwiGLU; the comparison is of the
+    contractions' throughput."""
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    from sparse_mixture_experts_05_b200.inputs import make_inputs
+
+    device = torch.device("cuda", 0)
+    w = workload(a.workload, a.tokens, a.experts)
+    T, d, d_ff, E, k = w.T, w.d, w.d_ff, w.E, w.k
+    R = T * k
+    if R % E:
+        raise SystemExit("--vs-cublas needs T*k divisible by E")
+    inp = make_inputs(R, d, d_ff, E, 1, w.seed, device=device)
+    xs = inp["x"]  # used directly as the expert-sorted rows, R/E per expert
+    W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
+    W13 = torch.cat([W1, W3], dim=2).contiguous()
+    off = torch.arange(0, R + 1, R // E, dtype=torch.int32, device=device)
+    shape = (T, d, d_ff, E, k)
+    h = torch.empty(R, d_ff, dtype=torch.bfloat16, device=device)
+    o = torch.empty(R, d, dtype=torch.float32, device=device)
+    ws = moe.workspace(moe.moe_expert_workspace_bytes(shape), device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    xb = xs.view(E, R // E, d)
+    hb = h.view(E, R // E, d_ff)
+
+    def ours():
+        moe.moe_expert_swiglu(shape, xs, off, W1, W3, W2, h=h, o=o, ws=ws)
+
+    def cublas():
+        torch.bmm(xb, W13)
+        torch.bmm(hb, W2)
+
+    for _ in range(a.warmup):
+        ours()
+        cublas()
+    torch.cuda.synchronize()
+    times = {"ours": [], "cublas": []}
+    clock = ClockSampler(0)
+    clock.start()
+    for i in range(a.steps):
+        for name, fn in (("ours", ours), ("cublas", cublas)):
+            flush.fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            times[name].append(e0.elapsed_time(e1))
+    clocks = clock.stop()
+    if moe.moe_read_device_status(ws) != moe.MOE_OK:
+        raise RuntimeError("device status error")
+    flops = 2.0 * R * d * 2 * d_ff + 2.0 * R * d_ff * d
+    med = {n: statistics.median(v) for n, v in times.items()}
+    print(json.dumps({
+        "metric": "expert GEMM TFLOP/s vs cuBLAS batched bf16 GEMMs (same shapes, alternating)",
+        "config": {"workload": workload_label(a), "rows_per_expert": R // E, "d": d,
+                   "d_ff": d_ff, "E": E},
+        "steps": a.steps, "warmup": a.warmup,
+        "ours_ms": round(med["ours"], 4), "cublas_ms": round(med["cublas"], 4),
+        "ours_tflops": round(flops / (med["ours"] / 1e3) / 1e12, 1),
+        "cublas_tflops": round(flops / (med["cublas"] / 1e3) / 1e12, 1),
+        "ours_over_cublas": round(med["cublas"] / med["ours"], 4),
+        "ours_ms_all": [round(t, 4) for t in times["ours"]],
+        "cublas_ms_all": [round(t, 4) for t in times["cublas"]],
+        "clocks": clocks}))
+
+
 def main(argv=None):
     a = parse(argv)
     if a.impl == "reference":
         run_reference(a)
+    elif a.vs_cublas:
+        vs_cublas(a)
     else:
         run_ours(a)
     return 0
