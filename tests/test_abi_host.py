@@ -111,6 +111,38 @@ def test_null_and_misaligned_pointers_are_rejected_without_launch():
                  None, None, good, ctypes.c_size_t(16), None) == moe.MOE_ERR_WORKSPACE
 
 
+def test_block_hostio_and_dispatch_reject_bad_arguments_on_host():
+    S = binding.MoeShape(64, 128, 256, 8, 2)
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    bad = P((1 << 20) + 8)
+    eps = ctypes.c_float(1e-5)
+    big = ctypes.c_size_t(1 << 30)
+    # block: a misaligned gamma, a negative eps, a NaN eps, a short workspace
+    assert _call("moe_block_forward", S, good, bad, eps, good, None, good, good, good, good, good,
+                 big, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_block_forward", S, good, good, ctypes.c_float(-1.0), good, None, good, good,
+                 good, good, good, big, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_block_forward", S, good, good, ctypes.c_float(float("nan")), good, None,
+                 good, good, good, good, good, big, None) == moe.MOE_ERR_INVALID_ARG
+    need = moe.moe_block_workspace_bytes((64, 128, 256, 8, 2))
+    assert _call("moe_block_forward", S, good, good, eps, good, None, good, good, good, good, good,
+                 ctypes.c_size_t(need - 1), None) == moe.MOE_ERR_WORKSPACE
+    # host I/O: missing host buffers, then a workspace one byte short
+    assert _call("moe_forward_hostio", S, None, good, None, good, good, good, good, good, big,
+                 None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_forward_hostio", S, good, good, None, good, good, good, None, good, big,
+                 None) == moe.MOE_ERR_INVALID_ARG
+    need = moe.moe_forward_hostio_workspace_bytes((64, 128, 256, 8, 2))
+    assert _call("moe_forward_hostio", S, good, good, None, good, good, good, good, good,
+                 ctypes.c_size_t(need - 1), None) == moe.MOE_ERR_WORKSPACE
+    # dispatch: no offsets, a misaligned x
+    assert _call("moe_dispatch", S, good, good, None, good, good, good, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_dispatch", S, good, bad, good, good, good, good, None) == \
+        moe.MOE_ERR_INVALID_ARG
+
+
 def test_aux_loss_rejects_bad_arguments_on_host():
     P = ctypes.c_void_p
     good = P(1 << 20)
