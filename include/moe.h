@@ -96,8 +96,9 @@ int moe_route(moe_shape s, const void* x, const void* Wg, const float* bias, int
               float* gate, float* logits, void* stream);
 
 /*
- * moe_dispatch -- per-expert token lists (dispatch of section "Алгоритм":
- * tok, slot = where(topk_idx == e), in ascending token order).
+ * moe_dispatch -- per-expert token lists (the dispatch step of section
+ * "Алгоритм": for each expert, the (token, slot) pairs whose top-k list names
+ * that expert, in ascending token order).
  *   idx [T,k] int32 (in), x [T,d] bf16 (in)
  *   offsets [E+1] int32: rows of expert e are offsets[e] .. offsets[e+1]-1 (out)
  *   perm_tok [T*k] int32: token of each sorted row (out)
@@ -158,7 +159,8 @@ int moe_expert_swiglu_stall_test(moe_shape s, const void* x_sorted, const int32_
 
 /*
  * moe_combine -- y[t] = sum over slots s (in slot order) of gate[t,s] * o[inv[t,s]]
- * (combine of section "Алгоритм": Y.index_add_(0, tok, W[tok,slot] * Expert_e(X[tok]))).
+ * (the combine step of section "Алгоритм": each token's output accumulates the
+ * gate-weighted outputs of the experts it was sent to, k terms per token).
  * Products and sums in float32 without fused multiply-add; y rounded to bf16.
  *   o [T*k,d] float, inv [T,k] int32, gate [T,k] float (in);  y [T,d] bf16 (out)
  * Slots with inv < 0 are skipped.
@@ -168,6 +170,10 @@ int moe_combine(moe_shape s, const float* o, const int32_t* inv, const float* ga
 
 /*
  * moe_forward -- the whole layer: route, dispatch, experts, combine.
+ * Page: the MoE equation of section "Прямой проход в формулах"
+ * (MoE(u) = sum_{i in S} w_i Expert_i(u)), computed in the order of section
+ * "Алгоритм" (route every token, then one pass per expert over its tokens,
+ * then k gate-weighted terms per token).
  *   x, Wg, bias (nullable), W1, W3, W2 as above (in);  y [T,d] bf16 (out)
  *   idx_out [T,k] int32, gate_out [T,k] float: copies of the routing, or NULL
  *   ws: >= moe_forward_workspace_bytes(s) bytes of device memory
@@ -179,6 +185,8 @@ int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, c
 /*
  * moe_forward_bias -- moe_forward with the biases of the expert Linear layers
  * (b1, b3 [E,d_ff], b2 [E,d] float, each nullable; see moe_expert_swiglu_bias).
+ * Page: section "Подсчёт параметров" (the teaching configuration puts a bias on
+ * every Linear, so each expert computes SiLU(u W1 + b1) (.) (u W3 + b3) W2 + b2).
  * The router bias is `bias`, as for moe_forward.
  */
 int moe_forward_bias(moe_shape s, const void* x, const void* Wg, const float* bias,
@@ -233,6 +241,23 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
                        size_t ws_bytes, void* stream);
 
 /*
+ * moe_forward_hostio_stall_test -- test hook for the error path of the chunked
+ * host-I/O pipeline (no counterpart on the pages).  Runs moe_forward_hostio with
+ * the expert kernels' TMA producer of token chunk `stall_chunk` (0 = first;
+ * batches of 2048+ tokens run as two chunks, smaller ones as one; a chunk index
+ * past the last stalls nothing) stopping after `stall_after` (>= 0) pipeline
+ * stages, and that chunk's device waits bounded by `timeout_ns` (1e3 .. 2e9).
+ * The status word is cleared once per call, before the first chunk, so
+ * moe_read_device_status(ws) reports MOE_ERR_DEVICE_TIMEOUT whichever chunk's
+ * wait expired.  y is then incomplete; the CUDA context stays usable.
+ */
+int moe_forward_hostio_stall_test(moe_shape s, const void* x_host, const void* Wg,
+                                  const float* bias, const void* W1, const void* W3,
+                                  const void* W2, void* y_host, void* ws, size_t ws_bytes,
+                                  int stall_chunk, int stall_after, uint64_t timeout_ns,
+                                  void* stream);
+
+/*
  * moe_aux_loss -- load-balancing auxiliary term of the router (Mixtral textbook
  * page, section "Load-balancing loss"):
  *     aux = E * sum_{s<k} sum_{i<E} f_{s,i} * P_i
@@ -263,7 +288,7 @@ int moe_aux_loss(moe_shape s, const float* logits, const int32_t* idx, const uin
  * caller still passes every input and the output y, all in device memory.
  *  - Limit: shapes with moe_forward_workspace_bytes(s) > 8 MiB are rejected
  *    with MOE_ERR_WORKSPACE before anything is launched (for d = 4096,
- *    d_ff = 14336, k = 2 that allows T <= 64 tokens: decode-sized batches).
+ *    d_ff = 14336, k = 2 that allows T <= 78 tokens: decode-sized batches).
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture begins.
@@ -273,7 +298,8 @@ int moe_aux_loss(moe_shape s, const float* logits, const int32_t* idx, const uin
  *    host threads, on one device) race on the array: serialise them.
  *  - device_status: nullable device int32; when given, it receives the call's
  *    status word (0, or nonzero after an expired device wait; see
- *    moe_read_device_status) once the call's work has run.
+ *    moe_read_device_status) once the call's work has run.  With T == 0 nothing
+ *    is launched except the write of 0 to device_status.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  */
 #define MOE_STATIC_SCRATCH_BYTES (8u << 20)

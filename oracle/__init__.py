@@ -6,7 +6,8 @@ module and shares no code with it.
 
 Every routine follows the Mixtral textbook page (llm-arch-research), section
 "Прямой проход в формулах" (the MoE equation) and section "Алгоритм" (the loop
-over experts with where/index_add); the C source cites the passage per routine.
+over experts, gathering each expert's tokens and accumulating the gate-weighted
+outputs back per token); the C source cites the passage per routine.
 
 Arrays are numpy: bf16 tensors travel as uint16 bit patterns.
 """

@@ -124,8 +124,8 @@ int orc_route(int T, int d, int E, int k, const uint16_t* x, const uint16_t* wg,
 }
 
 /* ---- dispatch ---------------------------------------------------------------
- * Section "Алгоритм": for expert e, (tok, slot) = where(topk_idx == e), read in
- * row-major order, i.e. by ascending token.  The per-expert lists are laid end
+ * Section "Алгоритм": for expert e, the (token, slot) pairs whose top-k list
+ * names e, read in row-major order, i.e. by ascending token.  The per-expert lists are laid end
  * to end: offsets[e] = number of (token, slot) entries routed to experts < e.
  *   offsets [E+1], perm_tok [T*k] (token of each sorted row),
  *   inv [T, k] (sorted row of each (token, slot)). */

@@ -29,7 +29,8 @@ EXPORTS = (
     "moe_status_string", "moe_check_shape", "moe_expert_workspace_bytes",
     "moe_forward_workspace_bytes", "moe_forward_hostio_workspace_bytes", "moe_route",
     "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_bias", "moe_expert_swiglu_stall_test",
-    "moe_combine", "moe_forward", "moe_forward_bias", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_static",
+    "moe_combine", "moe_forward", "moe_forward_bias", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_hostio_stall_test",
+    "moe_forward_static",
     "moe_aux_loss", "moe_block_workspace_bytes", "moe_block_forward", "moe_read_device_status",
 )
 
@@ -91,6 +92,9 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, Z, P, I, P]
         L.moe_forward_hostio.restype = I
         L.moe_forward_hostio.argtypes = [S, P, P, P, P, P, P, P, P, Z, P]
+        L.moe_forward_hostio_stall_test.restype = I
+        L.moe_forward_hostio_stall_test.argtypes = [S, P, P, P, P, P, P, P, P, Z, I, I,
+                                                    ctypes.c_uint64, P]
         L.moe_forward_static.restype = I
         L.moe_forward_static.argtypes = [S, P, P, P, P, P, P, P, P, P]
         L.moe_block_forward.restype = I
@@ -365,6 +369,31 @@ def moe_forward_hostio(shape, x_host, Wg, bias, W1, W3, W2, y_host, ws, stream=N
     _check("moe_forward_hostio",
            lib().moe_forward_hostio(_shape(shape), _p(x_host), _p(Wg), _p(bias), _p(W1), _p(W3),
                                     _p(W2), _p(y_host), _p(ws), ws.numel(), _stream(stream)))
+    return y_host
+
+
+def moe_forward_hostio_stall_test(shape, x_host, Wg, bias, W1, W3, W2, y_host, ws,
+                                  stall_chunk: int, stall_after: int, timeout_ns: int,
+                                  stream=None):
+    """moe_forward_hostio with the expert producer of token chunk `stall_chunk`
+    stopping after `stall_after` stages and that chunk's waits bounded by
+    `timeout_ns` (test of the error path of the chunked pipeline)."""
+    T, d, d_ff, E, k = shape
+    for name, t in (("x_host", x_host), ("y_host", y_host)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() \
+                or tuple(t.shape) != (T, d):
+            raise ValueError(f"{name} must be a contiguous CPU bf16 tensor of shape {(T, d)}")
+    _dev(Wg, "Wg", torch.bfloat16, (d, E))
+    _dev(bias, "bias", torch.float32, (E,))
+    _dev(W1, "W1", torch.bfloat16, (E, d, d_ff))
+    _dev(W3, "W3", torch.bfloat16, (E, d, d_ff))
+    _dev(W2, "W2", torch.bfloat16, (E, d_ff, d))
+    _dev(ws, "ws", torch.uint8)
+    _check("moe_forward_hostio_stall_test",
+           lib().moe_forward_hostio_stall_test(_shape(shape), _p(x_host), _p(Wg), _p(bias), _p(W1),
+                                               _p(W3), _p(W2), _p(y_host), _p(ws), ws.numel(),
+                                               int(stall_chunk), int(stall_after),
+                                               int(timeout_ns), _stream(stream)))
     return y_host
 
 

@@ -87,9 +87,6 @@ T* at(void* base, size_t off) {
 
 constexpr int kProfileEvents = 7;
 
-// Records events[i] (when given) between the launches: 0 before the router, 1
-// after it, 2 after the dispatch index kernel, 3 after the scatter, 4 after
-// GEMM1, 5 after GEMM2, 6 after the combine.
 // Biases of the expert Linear layers (each nullable): b1, b3 [E, d_ff], b2 [E, d].
 struct ExpertBias {
     const float* b1 = nullptr;
@@ -97,11 +94,23 @@ struct ExpertBias {
     const float* b2 = nullptr;
 };
 
+// Variations of one forward pass.
+struct FwdOptions {
+    const void* residual = nullptr;  // [T, d] bf16 added before the rounding of y (block edge)
+    ExpertBias eb;                   // expert Linear biases
+    int router_split = 0;            // router k-split (0: chosen for this T)
+    bool clear_status = true;        // the index kernel zeroes the status word first
+    int stall_after = -1;            // test hook: expert producer stops after this many stages
+    uint64_t timeout_ns = kDefaultWaitTimeoutNs;  // bound on every device wait
+};
+
+// Records events[i] (when given) between the launches: 0 before the router, 1
+// after it, 2 after the dispatch index kernel, 3 after the scatter, 4 after
+// GEMM1, 5 after GEMM2, 6 after the combine.
 int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                  const void* W1, const void* W3, const void* W2, void* y, int32_t* idx_out,
                  float* gate_out, void* ws, cudaStream_t st, void* const* events,
-                 const void* residual = nullptr, const ExpertBias& eb = ExpertBias{},
-                 int router_split = 0) {
+                 const FwdOptions& opt = FwdOptions{}) {
     auto mark = [&](int i) {
         return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
     };
@@ -116,20 +125,20 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     float* o = at<float>(ws, L.o);
     int* status = at<int>(ws, L.hdr);
     if (!mark(0)) return MOE_ERR_CUDA;
-    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, router_split);
+    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_split);
     if (rc) return rc;
     if (!mark(1)) return MOE_ERR_CUDA;
-    rc = launch_dispatch_index(s, idx, offsets, perm, inv, status, st);
+    rc = launch_dispatch_index(s, idx, offsets, perm, inv, opt.clear_status ? status : nullptr, st);
     if (rc) return rc;
     if (!mark(2)) return MOE_ERR_CUDA;
     rc = launch_dispatch_scatter(s, x, inv, xs, st);
     if (rc) return rc;
     if (!mark(3)) return MOE_ERR_CUDA;
-    rc = expert_gemms(s, xs, offsets, W1, W3, W2, h, o, status, kDefaultWaitTimeoutNs, -1, st,
-                      events ? events[4] : nullptr, eb.b1, eb.b3, eb.b2);
+    rc = expert_gemms(s, xs, offsets, W1, W3, W2, h, o, status, opt.timeout_ns, opt.stall_after,
+                      st, events ? events[4] : nullptr, opt.eb.b1, opt.eb.b3, opt.eb.b2);
     if (rc) return rc;
     if (!mark(5)) return MOE_ERR_CUDA;
-    rc = launch_combine(s, o, inv, gate, y, st, residual);
+    rc = launch_combine(s, o, inv, gate, y, st, opt.residual);
     if (rc) return rc;
     return mark(6) ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -188,6 +197,85 @@ CopyStreams* copy_streams() {
         per_device[dev] = cs;
     }
     return per_device[dev];
+}
+
+// moe_forward_hostio with an optional stall of the expert producer in chunk
+// `stall_chunk` (test hook; -1: none).  The status word is cleared once, by the
+// first chunk's index kernel: a later chunk must not erase an expired wait that
+// an earlier chunk recorded.
+int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const float* bias,
+                const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
+                size_t ws_bytes, cudaStream_t st, int stall_chunk, int stall_after,
+                uint64_t timeout_ns) {
+    int rc = check_shape(s);
+    if (rc || s.T == 0) return rc;
+    if (!x_host || !y_host || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) ||
+        !ok_ptr(W2) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_hostio_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    const size_t fwd = moe_forward_workspace_bytes(s);
+    const size_t io_bytes = (size_t)s.T * s.d * 2;
+    char* x_dev = static_cast<char*>(ws) + fwd;
+    char* y_dev = static_cast<char*>(ws) + fwd + align_up(io_bytes, 256);
+    auto chunk_opt = [&](int c) {
+        FwdOptions opt;
+        opt.clear_status = c == 0;
+        if (c == stall_chunk) {
+            opt.stall_after = stall_after;
+            opt.timeout_ns = timeout_ns;
+        }
+        return opt;
+    };
+    const int chunks = hostio_chunks(s.T);
+    if (chunks == 1) {
+        if (cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        rc = forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st,
+                          nullptr, chunk_opt(0));
+        if (rc) return rc;
+        if (cudaMemcpyAsync(y_host, y_dev, io_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    // Token chunks in a pipeline: the layer is independent per token, so chunk c
+    // computes (on `st`) while chunk c+1's x is still arriving and chunk c-1's y
+    // is leaving, on the two copy engines.  The result equals the unchunked
+    // layer bit for bit: no row's arithmetic depends on the other rows.
+    CopyStreams* cs = copy_streams();
+    if (!cs) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(cs->mu);
+    const int per = (s.T + chunks - 1) / chunks;
+    const int split = router_ksplit(s);  // the whole batch's: every chunk rounds alike
+    const size_t row_bytes = (size_t)s.d * 2;
+    bool ok = cudaEventRecord(cs->ev[0], st) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->up, cs->ev[0], 0) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->down, cs->ev[0], 0) == cudaSuccess;
+    for (int c = 0; ok && c < chunks; ++c) {
+        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
+        ok = cudaMemcpyAsync(x_dev + t0 * row_bytes, static_cast<const char*>(x_host) + t0 * row_bytes,
+                             (size_t)tn * row_bytes, cudaMemcpyHostToDevice, cs->up) == cudaSuccess &&
+             cudaEventRecord(cs->ev[1 + c], cs->up) == cudaSuccess;
+    }
+    for (int c = 0; ok && c < chunks; ++c) {
+        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
+        moe_shape sc = s;
+        sc.T = tn;
+        FwdOptions opt = chunk_opt(c);
+        opt.router_split = split;
+        ok = cudaStreamWaitEvent(st, cs->ev[1 + c], 0) == cudaSuccess &&
+             forward_impl(sc, x_dev + t0 * row_bytes, Wg, bias, W1, W3, W2, y_dev + t0 * row_bytes,
+                          nullptr, nullptr, ws, st, nullptr, opt) == MOE_OK &&
+             cudaEventRecord(cs->ev[1 + kMaxHostioChunks + c], st) == cudaSuccess &&
+             cudaStreamWaitEvent(cs->down, cs->ev[1 + kMaxHostioChunks + c], 0) == cudaSuccess &&
+             cudaMemcpyAsync(static_cast<char*>(y_host) + t0 * row_bytes, y_dev + t0 * row_bytes,
+                             (size_t)tn * row_bytes, cudaMemcpyDeviceToHost,
+                             cs->down) == cudaSuccess;
+    }
+    // join: the caller's stream waits for the last copy back
+    const int last = 1 + 2 * kMaxHostioChunks;
+    ok = ok && cudaEventRecord(cs->ev[last], cs->down) == cudaSuccess &&
+         cudaStreamWaitEvent(st, cs->ev[last], 0) == cudaSuccess;
+    return ok ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -336,12 +424,12 @@ int moe_forward_bias(moe_shape s, const void* x, const void* Wg, const float* bi
         !ok_opt(gate_out) || !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_forward_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
-    ExpertBias eb;
-    eb.b1 = b1;
-    eb.b3 = b3;
-    eb.b2 = b2;
+    FwdOptions opt;
+    opt.eb.b1 = b1;
+    opt.eb.b3 = b3;
+    opt.eb.b2 = b2;
     return forward_impl(s, x, Wg, bias, W1, W3, W2, y, idx_out, gate_out, ws,
-                        static_cast<cudaStream_t>(stream), nullptr, nullptr, eb);
+                        static_cast<cudaStream_t>(stream), nullptr, opt);
 }
 
 int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float* bias,
@@ -372,86 +460,47 @@ int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, 
     void* u = static_cast<char*>(ws) + moe_forward_workspace_bytes(s);
     rc = launch_rmsnorm(s, U, gamma, eps, u, st);
     if (rc) return rc;
-    return forward_impl(s, u, Wg, bias, W1, W3, W2, H, nullptr, nullptr, ws, st, nullptr, U);
+    FwdOptions opt;
+    opt.residual = U;
+    return forward_impl(s, u, Wg, bias, W1, W3, W2, H, nullptr, nullptr, ws, st, nullptr, opt);
 }
 
 int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const float* bias,
                        const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
                        size_t ws_bytes, void* stream) {
-    int rc = check_shape(s);
-    if (rc || s.T == 0) return rc;
-    if (!x_host || !y_host || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) ||
-        !ok_ptr(W2) || !ok_ptr(ws))
-        return MOE_ERR_INVALID_ARG;
-    if (ws_bytes < moe_forward_hostio_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t fwd = moe_forward_workspace_bytes(s);
-    const size_t io_bytes = (size_t)s.T * s.d * 2;
-    char* x_dev = static_cast<char*>(ws) + fwd;
-    char* y_dev = static_cast<char*>(ws) + fwd + align_up(io_bytes, 256);
-    const int chunks = hostio_chunks(s.T);
-    if (chunks == 1) {
-        if (cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        rc = forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st,
-                          nullptr);
-        if (rc) return rc;
-        if (cudaMemcpyAsync(y_host, y_dev, io_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        return MOE_OK;
-    }
-    // Token chunks in a pipeline: the layer is independent per token, so chunk c
-    // computes (on `st`) while chunk c+1's x is still arriving and chunk c-1's y
-    // is leaving, on the two copy engines.  The result equals the unchunked
-    // layer bit for bit: no row's arithmetic depends on the other rows.
-    CopyStreams* cs = copy_streams();
-    if (!cs) return MOE_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(cs->mu);
-    const int per = (s.T + chunks - 1) / chunks;
-    const int split = router_ksplit(s);  // the whole batch's: every chunk rounds alike
-    const size_t row_bytes = (size_t)s.d * 2;
-    bool ok = cudaEventRecord(cs->ev[0], st) == cudaSuccess &&
-              cudaStreamWaitEvent(cs->up, cs->ev[0], 0) == cudaSuccess &&
-              cudaStreamWaitEvent(cs->down, cs->ev[0], 0) == cudaSuccess;
-    for (int c = 0; ok && c < chunks; ++c) {
-        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
-        ok = cudaMemcpyAsync(x_dev + t0 * row_bytes, static_cast<const char*>(x_host) + t0 * row_bytes,
-                             (size_t)tn * row_bytes, cudaMemcpyHostToDevice, cs->up) == cudaSuccess &&
-             cudaEventRecord(cs->ev[1 + c], cs->up) == cudaSuccess;
-    }
-    for (int c = 0; ok && c < chunks; ++c) {
-        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
-        moe_shape sc = s;
-        sc.T = tn;
-        ok = cudaStreamWaitEvent(st, cs->ev[1 + c], 0) == cudaSuccess &&
-             forward_impl(sc, x_dev + t0 * row_bytes, Wg, bias, W1, W3, W2, y_dev + t0 * row_bytes,
-                          nullptr, nullptr, ws, st, nullptr, nullptr, ExpertBias{},
-                          split) == MOE_OK &&
-             cudaEventRecord(cs->ev[1 + kMaxHostioChunks + c], st) == cudaSuccess &&
-             cudaStreamWaitEvent(cs->down, cs->ev[1 + kMaxHostioChunks + c], 0) == cudaSuccess &&
-             cudaMemcpyAsync(static_cast<char*>(y_host) + t0 * row_bytes, y_dev + t0 * row_bytes,
-                             (size_t)tn * row_bytes, cudaMemcpyDeviceToHost,
-                             cs->down) == cudaSuccess;
-    }
-    // join: the caller's stream waits for the last copy back
-    const int last = 1 + 2 * kMaxHostioChunks;
-    ok = ok && cudaEventRecord(cs->ev[last], cs->down) == cudaSuccess &&
-         cudaStreamWaitEvent(st, cs->ev[last], 0) == cudaSuccess;
-    return ok ? MOE_OK : MOE_ERR_CUDA;
+    return hostio_impl(s, x_host, Wg, bias, W1, W3, W2, y_host, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream), -1, -1, kDefaultWaitTimeoutNs);
+}
+
+int moe_forward_hostio_stall_test(moe_shape s, const void* x_host, const void* Wg,
+                                  const float* bias, const void* W1, const void* W3,
+                                  const void* W2, void* y_host, void* ws, size_t ws_bytes,
+                                  int stall_chunk, int stall_after, uint64_t timeout_ns,
+                                  void* stream) {
+    if (stall_chunk < 0 || stall_after < 0) return MOE_ERR_INVALID_ARG;
+    if (timeout_ns < 1000 || timeout_ns > kDefaultWaitTimeoutNs) return MOE_ERR_INVALID_ARG;
+    return hostio_impl(s, x_host, Wg, bias, W1, W3, W2, y_host, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream), stall_chunk, stall_after, timeout_ns);
 }
 
 int moe_forward_static(moe_shape s, const void* x, const void* Wg, const float* bias,
                        const void* W1, const void* W3, const void* W2, void* y,
                        int32_t* device_status, void* stream) {
     int rc = check_shape(s);
-    if (rc || s.T == 0) return rc;
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (s.T == 0) {  // nothing to compute; the status word still reports "fine"
+        if (!ok_opt(device_status)) return MOE_ERR_INVALID_ARG;
+        if (device_status && cudaMemsetAsync(device_status, 0, sizeof(int32_t), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
     if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
         !ok_ptr(y) || !ok_opt(device_status))
         return MOE_ERR_INVALID_ARG;
     if (moe_forward_workspace_bytes(s) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
     void* ws = static_scratch_address();
     if (!ws) return MOE_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     // forward_impl zeroes the status word (first word of the scratch) itself and
     // overwrites every other scratch byte it reads, so nothing else needs clearing.
     rc = forward_impl(s, x, Wg, bias, W1, W3, W2, y, nullptr, nullptr, ws, st, nullptr);

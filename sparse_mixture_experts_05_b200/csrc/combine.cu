@@ -1,7 +1,7 @@
 // combine.cu -- gate-weighted un-permute of the expert outputs.
 //
-// Mixtral textbook page, section "Алгоритм": Y.index_add_(0, tok,
-// W[tok, slot] * Expert_e(X[tok])) -- every token receives exactly k terms.
+// Mixtral textbook page, section "Алгоритм": each token's output accumulates
+// the gate-weighted outputs of the experts it was routed to -- exactly k terms.
 // Each token's terms are gathered from their sorted rows and added in slot
 // order: products and sums are separately rounded float32 operations (no fused
 // multiply-add), so the result does not depend on scheduling and needs no

@@ -1,8 +1,8 @@
 // dispatch.cu -- per-expert token lists and the expert-sorted copy of x.
 //
-// Mixtral textbook page, section "Алгоритм": for each expert e,
-// (tok, slot) = where(topk_idx == e) lists the tokens that chose e in ascending
-// token order, and the expert runs once over X[tok].  Here the lists of all
+// Mixtral textbook page, section "Алгоритм": for each expert e, the
+// (token, slot) pairs whose top-k list names e, taken in ascending token order,
+// and the expert runs once over those tokens' rows.  Here the lists of all
 // experts are laid end to end (offsets[e] .. offsets[e+1]-1), which is the order
 // an exclusive scan of the per-expert counts produces.
 //

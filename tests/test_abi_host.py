@@ -143,6 +143,36 @@ def test_block_hostio_and_dispatch_reject_bad_arguments_on_host():
         moe.MOE_ERR_INVALID_ARG
 
 
+def test_hostio_stall_hook_rejects_bad_arguments_on_host():
+    S = binding.MoeShape(64, 128, 256, 8, 2)
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    big = ctypes.c_size_t(1 << 30)
+    t = ctypes.c_uint64(10 ** 6)
+    assert _call("moe_forward_hostio_stall_test", S, good, good, None, good, good, good, good,
+                 good, big, -1, 1, t, None) == moe.MOE_ERR_INVALID_ARG      # negative chunk
+    assert _call("moe_forward_hostio_stall_test", S, good, good, None, good, good, good, good,
+                 good, big, 0, -1, t, None) == moe.MOE_ERR_INVALID_ARG      # negative stage count
+    assert _call("moe_forward_hostio_stall_test", S, good, good, None, good, good, good, good,
+                 good, big, 0, 1, ctypes.c_uint64(10), None) == moe.MOE_ERR_INVALID_ARG
+    assert _call("moe_forward_hostio_stall_test", S, None, good, None, good, good, good, good,
+                 good, big, 0, 1, t, None) == moe.MOE_ERR_INVALID_ARG      # no host x
+
+
+def test_static_scratch_limit_is_78_tokens_at_the_mixtral_widths():
+    """The static scratch holds the whole forward workspace of up to 78 tokens
+    at d = 4096, d_ff = 14336, k = 2; 79 tokens are rejected before any launch."""
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    assert moe.moe_forward_workspace_bytes((78, 4096, 14336, 8, 2)) <= binding.MOE_STATIC_SCRATCH_BYTES
+    assert moe.moe_forward_workspace_bytes((79, 4096, 14336, 8, 2)) > binding.MOE_STATIC_SCRATCH_BYTES
+    assert _call("moe_forward_static", binding.MoeShape(79, 4096, 14336, 8, 2), good, good, None,
+                 good, good, good, good, None, None) == moe.MOE_ERR_WORKSPACE
+    # T = 0 launches nothing (no status pointer given)
+    assert _call("moe_forward_static", binding.MoeShape(0, 4096, 14336, 8, 2), None, None, None,
+                 None, None, None, None, None, None) == moe.MOE_OK
+
+
 def test_aux_loss_rejects_bad_arguments_on_host():
     P = ctypes.c_void_p
     good = P(1 << 20)

@@ -137,6 +137,33 @@ def test_expert_swiglu(name):
                       row_expert, inp["W1"], inp["W3"], inp["W2"], h_ref, o_ref)
 
 
+def test_expert_swiglu_extreme_gate_inputs():
+    """SiLU's tails: W1 scaled by 32 and W3 by 4 (powers of two, so the bf16
+    weights stay exact) make a = x W1 span about +-100 and b = x W3 about +-12,
+    including many a < -87.3, where 1 + e^-a exceeds 2^126.  h must still meet
+    the one-bf16-ulp-plus-accumulation bound against the oracle there."""
+    inp = make_inputs(512, 256, 512, 8, 2, seed=47)
+    inp["W1"] = (inp["W1"].float() * 32).to(torch.bfloat16)
+    inp["W3"] = (inp["W3"].float() * 4).to(torch.bfloat16)
+    T, d, d_ff, E, k = inp["shape"]
+    o_idx, _, _ = oracle.route(inp["x"], inp["Wg"], E, k)
+    r_off, r_perm, _ = oracle.dispatch(o_idx, E)
+    xs = oracle.gather(inp["x"], r_perm)
+    h_ref, o_ref = oracle.expert(xs, r_off, inp["W1"], inp["W3"], inp["W2"])
+    row_expert = np.searchsorted(r_off, np.arange(T * k), side="right") - 1
+    xv = oracle.bf16_to_f64(xs)
+    a = np.concatenate([xv[row_expert == e] @ bf16_values(inp["W1"][e]) for e in range(E)])
+    assert a.min() < -100 and a.max() > 100
+    assert np.sum((a < -87.3) & (a > -104)) > 100   # the region the plain form gets wrong
+    dev = to_dev(inp)
+    xs_t = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16).cuda()
+    h, o, ws = moe.moe_expert_swiglu(inp["shape"], xs_t, torch.from_numpy(r_off).cuda(),
+                                     dev["W1"], dev["W3"], dev["W2"])
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    check_expert_rows(bf16_values(h), o.cpu().numpy().astype(np.float64), xv, row_expert,
+                      inp["W1"], inp["W3"], inp["W2"], h_ref, o_ref)
+
+
 @pytest.mark.parametrize("name", ALL)
 def test_combine(name):
     inp = _inputs(name)
@@ -250,6 +277,31 @@ def test_hostio_token_chunks_equal_the_whole_batch(T):
     torch.cuda.synchronize()
     assert torch.equal(y_dev.cpu(), y_host)
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
+
+
+@pytest.mark.parametrize("T,stall_chunk", [(2048, 0), (2048, 1), (300, 0)],
+                         ids=["first-of-two-chunks", "second-of-two-chunks", "one-chunk"])
+def test_hostio_reports_a_timeout_in_any_chunk(T, stall_chunk):
+    """The host-I/O pipeline runs large batches as token chunks on one
+    workspace; a wait that expires in an earlier chunk must not be cleared by a
+    later one.  The stalled chunk's producer stops after one stage (2 ms bound):
+    the status must read MOE_ERR_DEVICE_TIMEOUT, and a normal call afterwards on
+    the same workspace must be correct and report MOE_OK."""
+    inp = make_inputs(T, 256, 256, 8, 2, seed=45, bias=True)
+    dev = to_dev(inp)
+    shape = inp["shape"]
+    args = (dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    x_host = inp["x"].clone().pin_memory()
+    y_host = torch.zeros(T, 256, dtype=torch.bfloat16).pin_memory()
+    ws = moe.workspace(moe.moe_forward_hostio_workspace_bytes(shape), "cuda")
+    moe.moe_forward_hostio_stall_test(shape, x_host, *args, y_host, ws, stall_chunk=stall_chunk,
+                                      stall_after=1, timeout_ns=2_000_000)
+    assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    moe.moe_forward_hostio(shape, x_host, *args, y_host, ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    y_dev = moe.moe_forward(shape, dev["x"], *args)
+    torch.cuda.synchronize()
+    assert torch.equal(y_dev.cpu(), y_host)
 
 
 @pytest.mark.parametrize("T", [8, 64, 300], ids=["tiny-batch", "single-cta", "cta-pair"])

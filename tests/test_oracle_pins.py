@@ -313,7 +313,7 @@ def test_bf16_storage_of_h_stays_within_rounding_budget():
 
 
 def test_combine_slot_order_equals_expert_order():
-    """index_add_ over experts (section "Алгоритм") adds a token's terms in expert
+    """Accumulating over experts (section "Алгоритм") adds a token's terms in expert
     order; slot order gives the same value because both products are formed
     before a single addition of two terms (k = 2)."""
     rng = np.random.default_rng(8)
