@@ -57,7 +57,7 @@ def parse(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the decode-workload line added to the prefill run")
+                    help="skip the extras and the decode and skew objects of the prefill run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--tokens", type=int, default=None,
@@ -315,10 +315,13 @@ def timed_loop(ctx, steps, pg, device, clock, profiled):
     return step_ms, parts, outer0.elapsed_time(outer1), clocks
 
 
-def extras_loop(ctx, steps, device):
-    """The widened entry points on the same batch (each timed like the plain step,
-    L2 flushed before each call): the block with its edges, the layer with expert
-    biases, and the load-balancing term on the router's logits."""
+def extras_loop(ctx, steps, device, local):
+    """The widened entry points on the same batch, interleaved step by step with
+    the plain layer so that all see the same clocks and power state (L2 flushed
+    before every call, nvidia-smi sampled throughout): the block with its edges,
+    the layer with expert biases, and the load-balancing term on the router's
+    logits.  Reports each one's mean time and its difference from the plain
+    layer measured in the same loop."""
     import torch
 
     import sparse_mixture_experts_05_b200 as moe
@@ -335,29 +338,78 @@ def extras_loop(ctx, steps, device):
     H = torch.empty(T, d, dtype=torch.bfloat16, device=device)
     idx, _, logits = moe.moe_route(shape, x, Wg, bias, want_logits=True)
     calls = {
+        "plain_ms": lambda: moe.moe_forward(shape, x, Wg, bias, W1, W3, W2, y=ctx["y"],
+                                            ws=ctx["ws"]),
         "block_forward_ms": lambda: moe.moe_block_forward(shape, x, gamma, Wg, bias, W1, W3, W2,
                                                           H=H, ws=ws_b),
         "forward_bias_ms": lambda: moe.moe_forward_bias(shape, x, Wg, bias, W1, W3, W2, eb,
                                                         y=ctx["y"], ws=ctx["ws"]),
         "aux_loss_ms": lambda: moe.moe_aux_loss(shape, logits, idx),
     }
-    out = {}
-    for name, call in calls.items():
+    for call in calls.values():
         for _ in range(3):
             call()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)]
-        for i in range(steps):
+    torch.cuda.synchronize()
+    times = {name: [] for name in calls}
+    clock = ClockSampler(local)
+    clock.start()
+    for i in range(steps):
+        for name, call in calls.items():
             ctx["flush"].fill_(i & 0xFF)
-            evs[i][0].record()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
             call()
-            evs[i][1].record()
-        torch.cuda.synchronize()
-        out[name] = round(statistics.mean(a.elapsed_time(b) for a, b in evs), 4)
+            e1.record()
+            e1.synchronize()
+            times[name].append(e0.elapsed_time(e1))
+    clocks = clock.stop()
     if moe.moe_read_device_status(ws_b) != moe.MOE_OK:
         raise RuntimeError("device status error in the block forward")
-    out["note"] = ("same batch; block = RMSNorm + layer + residual; bias = expert Linear "
-                   "biases b1, b3, b2; aux = load-balancing term over the T x E logits")
+    out = {name: round(statistics.mean(v), 4) for name, v in times.items()}
+    out["block_minus_plain_ms"] = round(out["block_forward_ms"] - out["plain_ms"], 4)
+    out["bias_minus_plain_ms"] = round(out["forward_bias_ms"] - out["plain_ms"], 4)
+    out["clocks"] = clocks
+    out["note"] = ("same batch, calls interleaved step by step (plain, block, bias, aux); block = "
+                   "RMSNorm + layer + residual; bias = expert Linear biases b1, b3, b2; aux = "
+                   "load-balancing term over the T x E logits")
+    return out
+
+
+def secondary_workload(name, steps, warmup, device, rank, local, pg, peaks):
+    """A second workload timed like the main one (plain pass with clocks, then the
+    profiled pass for the kernel split) and summarised as an object of the line."""
+    w_steps = steps
+    ctx = time_workload(name, w_steps, warmup, device, rank)
+    ms, _, _, clocks = timed_loop(ctx, w_steps, pg, device, ClockSampler(local), profiled=False)
+    mean = reduce_max(pg, statistics.mean(ms), device)
+    pms, parts, _, _ = timed_loop(ctx, w_steps, pg, device, None, profiled=True)
+    pmean = reduce_max(pg, statistics.mean(pms), device)
+    alg = algorithmic(ctx["shape"], ctx["counts"])
+    gemm = parts["gemm1_swiglu"] + parts["gemm2_down"]
+    T = ctx["shape"][0]
+    world = 1 if pg is None else pg.get_world_size()
+    out = {"workload": WORKLOAD_NAMES[name], "tokens_per_s": round(T * world / (mean / 1e3), 1),
+           "ms_per_step": round(mean, 4), "steps": w_steps,
+           "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
+           "ms_per_step_profiled": round(pmean, 4), "expert_rows": ctx["counts"],
+           "clocks": clocks}
+    if name == "decode":
+        gbs = alg["bytes_experts_decode"] / (gemm / 1000) / 1e9
+        out.update({"experts_gbs": round(gbs, 1),
+                    "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                    "frac_of_spec_8000": round(gbs / SPEC_HBM_GBS, 4),
+                    "layer_gbs": round((alg["bytes_experts_decode"] + alg["bytes_router"]) /
+                                       (mean / 1000) / 1e9, 1)})
+    else:
+        tf = (alg["flops_gemm1"] + alg["flops_gemm2"]) / (gemm / 1000) / 1e12
+        out.update({"experts_tflops": round(tf, 1),
+                    "frac_of_measured_bf16": round(tf / peaks["bf16_tflops"], 4),
+                    "frac_of_spec_2250": round(tf / SPEC_BF16_TFLOPS, 4),
+                    "layer_tflops": round(alg["flops_total"] / (mean / 1000) / 1e12, 1)})
+    del ctx
+    import torch
+    torch.cuda.empty_cache()
     return out
 
 
@@ -495,34 +547,17 @@ def run_ours(a):
         "bracket_ms_incl_flush": round(bracket_ms, 3),
     }
     if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
-        line["extras"] = extras_loop(ctx, a.steps, device)
+        line["extras"] = extras_loop(ctx, a.steps, device, local)
     del ctx
     torch.cuda.empty_cache()
 
     if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
         # a decode step is ~0.5 ms: time at least 40 of them so the mean is stable
-        d_steps = max(a.steps, 40)
-        dctx = time_workload("decode", d_steps, a.warmup, device, rank)
-        d_ms, _, _, d_clocks = timed_loop(dctx, d_steps, pg, device, ClockSampler(local),
-                                          profiled=False)
-        d_mean = reduce_max(pg, statistics.mean(d_ms), device)
-        d_pms, d_parts, _, _ = timed_loop(dctx, d_steps, pg, device, None, profiled=True)
-        d_pmean = reduce_max(pg, statistics.mean(d_pms), device)
-        d_alg = algorithmic(dctx["shape"], dctx["counts"])
-        d_gemm = d_parts["gemm1_swiglu"] + d_parts["gemm2_down"]
-        d_gbs = d_alg["bytes_experts_decode"] / (d_gemm / 1000) / 1e9
-        line["decode"] = {
-            "workload": WORKLOAD_NAMES["decode"], "tokens_per_s": round(16 * world / (d_mean / 1e3), 1),
-            "ms_per_step": round(d_mean, 4), "steps": d_steps,
-            "experts_gbs": round(d_gbs, 1), "frac_of_measured_hbm": round(d_gbs / peaks["hbm_gbs"], 4),
-            "frac_of_spec_8000": round(d_gbs / SPEC_HBM_GBS, 4),
-            "layer_gbs": round((d_alg["bytes_experts_decode"] + d_alg["bytes_router"]) /
-                               (d_mean / 1000) / 1e9, 1),
-            "kernel_ms": {k_: round(v, 4) for k_, v in d_parts.items()},
-            "ms_per_step_profiled": round(d_pmean, 4),
-            "expert_rows": dctx["counts"], "clocks": d_clocks}
-        del dctx
-        torch.cuda.empty_cache()
+        line["decode"] = secondary_workload("decode", max(a.steps, 40), a.warmup, device, rank,
+                                            local, pg, peaks)
+        # the skewed prefill (T = 16384, biased router): ~9 ms a step
+        line["skew"] = secondary_workload("skew", min(a.steps, 10), a.warmup, device, rank,
+                                          local, pg, peaks)
 
     if world == 1 and rank == 0 and not a.no_cpu_baseline:
         from sparse_mixture_experts_05_b200.inputs import make_inputs

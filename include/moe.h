@@ -228,8 +228,10 @@ int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, 
  * copies y back; everything is ordered after earlier work on `stream`, and
  * `stream` is ordered after the last copy, so the caller synchronises `stream`
  * before reading y.  Weights stay on the device.  Batches of 2048 tokens or
- * more are split into two token halves whose copies run on two library-owned
- * copy streams (created once per device) while the other half computes:
+ * more are split into three token chunks (T/8 rounded down to a multiple of 64
+ * tokens, the rest, and T/8 again) whose copies run on two library-owned copy
+ * streams (created once per device) while the other chunks compute, so only
+ * the first chunk's upload and the last chunk's download are not overlapped:
  * the layer is independent per token, so y is the same bit for bit.  Calls
  * from several host threads on one device are enqueued one at a time.
  *   ws: >= moe_forward_workspace_bytes(s) + T*d*2 (x staging) + T*d*2 (y staging)
@@ -244,7 +246,7 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
  * moe_forward_hostio_stall_test -- test hook for the error path of the chunked
  * host-I/O pipeline (no counterpart on the pages).  Runs moe_forward_hostio with
  * the expert kernels' TMA producer of token chunk `stall_chunk` (0 = first;
- * batches of 2048+ tokens run as two chunks, smaller ones as one; a chunk index
+ * batches of 2048+ tokens run as three chunks, smaller ones as one; a chunk index
  * past the last stalls nothing) stopping after `stall_after` (>= 0) pipeline
  * stages, and that chunk's device waits bounded by `timeout_ns` (1e3 .. 2e9).
  * The status word is cleared once per call, before the first chunk, so

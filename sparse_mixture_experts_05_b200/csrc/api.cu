@@ -98,7 +98,7 @@ struct ExpertBias {
 struct FwdOptions {
     const void* residual = nullptr;  // [T, d] bf16 added before the rounding of y (block edge)
     ExpertBias eb;                   // expert Linear biases
-    int router_split = 0;            // router k-split (0: chosen for this T)
+    int router_cluster = 0;          // router cluster size, fixing its k split (0: chosen for this T)
     bool clear_status = true;        // the index kernel zeroes the status word first
     int stall_after = -1;            // test hook: expert producer stops after this many stages
     uint64_t timeout_ns = kDefaultWaitTimeoutNs;  // bound on every device wait
@@ -125,7 +125,7 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     float* o = at<float>(ws, L.o);
     int* status = at<int>(ws, L.hdr);
     if (!mark(0)) return MOE_ERR_CUDA;
-    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_split);
+    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_cluster);
     if (rc) return rc;
     if (!mark(1)) return MOE_ERR_CUDA;
     rc = launch_dispatch_index(s, idx, offsets, perm, inv, opt.clear_status ? status : nullptr, st);
@@ -166,11 +166,26 @@ void* static_scratch_address() {
     return addr[dev];
 }
 
-// moe_forward_hostio splits batches of 2048+ tokens into two halves whose copies
-// overlap the other half's computation.  (Four chunks measured slower: at 1024
-// tokens the down projection's CTA-pair tiles fill only 2.2 of 3 rounds.)
-constexpr int kMaxHostioChunks = 2;
-int hostio_chunks(int T) { return T >= 2048 ? 2 : 1; }
+// moe_forward_hostio splits batches of 2048+ tokens into three token chunks:
+// a small first chunk (T/8 rounded down to 64 tokens), the bulk, and a small
+// last chunk of the same size.  Copies run ahead of the computation (a token's
+// 8 KB cross the host link faster than the layer processes it), so only the
+// first chunk's upload and the last chunk's download are exposed; keeping those
+// chunks small shortens both, while the bulk keeps the GEMM tiles full.
+// (Two equal halves exposed 16 MiB each way at T = 4096; four equal chunks
+// measured slower, the down projection's tiles filling fewer rounds.)
+constexpr int kMaxHostioChunks = 3;
+int hostio_chunks(int T, int (&sizes)[kMaxHostioChunks]) {
+    if (T < 2048) {
+        sizes[0] = T;
+        return 1;
+    }
+    const int edge = (T / 8) / 64 * 64;
+    sizes[0] = edge;
+    sizes[1] = T - 2 * edge;
+    sizes[2] = edge;
+    return 3;
+}
 
 // Two copy streams (host->device, device->host) and the events that order them
 // against the caller's stream; created once per device and kept for the life
@@ -226,7 +241,8 @@ int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const fl
         }
         return opt;
     };
-    const int chunks = hostio_chunks(s.T);
+    int sizes[kMaxHostioChunks];
+    const int chunks = hostio_chunks(s.T, sizes);
     if (chunks == 1) {
         if (cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -244,24 +260,25 @@ int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const fl
     CopyStreams* cs = copy_streams();
     if (!cs) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(cs->mu);
-    const int per = (s.T + chunks - 1) / chunks;
-    const int split = router_ksplit(s);  // the whole batch's: every chunk rounds alike
+    int start[kMaxHostioChunks + 1] = {0};
+    for (int c = 0; c < chunks; ++c) start[c + 1] = start[c] + sizes[c];
+    const int split = router_cluster(s);  // the whole batch's: every chunk rounds alike
     const size_t row_bytes = (size_t)s.d * 2;
     bool ok = cudaEventRecord(cs->ev[0], st) == cudaSuccess &&
               cudaStreamWaitEvent(cs->up, cs->ev[0], 0) == cudaSuccess &&
               cudaStreamWaitEvent(cs->down, cs->ev[0], 0) == cudaSuccess;
     for (int c = 0; ok && c < chunks; ++c) {
-        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
+        const int t0 = start[c], tn = sizes[c];
         ok = cudaMemcpyAsync(x_dev + t0 * row_bytes, static_cast<const char*>(x_host) + t0 * row_bytes,
                              (size_t)tn * row_bytes, cudaMemcpyHostToDevice, cs->up) == cudaSuccess &&
              cudaEventRecord(cs->ev[1 + c], cs->up) == cudaSuccess;
     }
     for (int c = 0; ok && c < chunks; ++c) {
-        const int t0 = c * per, tn = std::min(s.T, t0 + per) - t0;
+        const int t0 = start[c], tn = sizes[c];
         moe_shape sc = s;
         sc.T = tn;
         FwdOptions opt = chunk_opt(c);
-        opt.router_split = split;
+        opt.router_cluster = split;
         ok = cudaStreamWaitEvent(st, cs->ev[1 + c], 0) == cudaSuccess &&
              forward_impl(sc, x_dev + t0 * row_bytes, Wg, bias, W1, W3, W2, y_dev + t0 * row_bytes,
                           nullptr, nullptr, ws, st, nullptr, opt) == MOE_OK &&

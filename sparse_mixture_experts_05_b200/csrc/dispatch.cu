@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
                  int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
                  int32_t* __restrict__ inv, int* status_to_clear) {
     __shared__ int s_pos[kIndexWarps][kMaxExperts + 1];  // counts, then next positions
+    __shared__ int s_total[kMaxExperts];                  // rows per expert
+    __shared__ int s_base[kMaxExperts];                   // first sorted row of each expert
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
@@ -76,29 +78,38 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
     }
     __syncthreads();
 
-    // offsets and per-warp starting positions (warp 0, lane = expert)
-    if (warp == 0) {
-        int total = 0;
-        if (lane < E)
-            for (int w = 0; w < kIndexWarps; ++w) {
-                const int c = s_pos[w][lane];
-                s_pos[w][lane] = total;  // position of this warp's first row of expert `lane`, relative
-                total += c;
-            }
-        // exclusive scan of the totals over experts
-        int incl = total;
+    // offsets and per-warp starting positions: warp e scans expert e's counts
+    // over the 32 warps (lane = warp), then warp 0 scans the experts' totals
+    {
+        int excl_w = 0;
+        if (warp < E) {
+            const int c = s_pos[lane][warp];
+            int incl = c;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += o;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            excl_w = incl - c;  // rows of expert `warp` in warps before `lane`
+            if (lane == 31) s_total[warp] = incl;
         }
-        const int excl = incl - total;
-        if (lane < E) {
-            offsets[lane] = excl;
-            for (int w = 0; w < kIndexWarps; ++w) s_pos[w][lane] += excl;
+        __syncthreads();
+        if (warp == 0) {
+            const int total = lane < E ? s_total[lane] : 0;
+            int incl = total;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            if (lane < E) {
+                s_base[lane] = incl - total;
+                offsets[lane] = incl - total;
+            }
+            if (lane == 31) offsets[E] = incl;
         }
-        const int all = __shfl_sync(0xffffffffu, incl, 31);
-        if (lane == 0) offsets[E] = all;
+        __syncthreads();
+        if (warp < E) s_pos[lane][warp] = s_base[warp] + excl_w;
     }
     __syncthreads();
 

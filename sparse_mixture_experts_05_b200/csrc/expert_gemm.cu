@@ -217,13 +217,14 @@ __device__ __forceinline__ float silu_times(float a, float b) {
     return a * sigma * b;
 }
 
-// GEMM1 epilogue of one TMEM lane (= one row): columns [0, hcols) hold
-// a = x W1, columns [hcols, 2 hcols) hold b = x W3 for the same output columns;
-// h = SiLU(a) * b (silu_times).  With `tma` the warp's 32 rows go
-// out through `map` (bf16, 64-byte rows, 64-byte swizzle) at (x0 + c, y0).
-// ba / bb (nullable) are the biases of the tile's first column for a and b.
-__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, bool tma,
-                                                __nv_bfloat16* hrow, int hcols,
+// GEMM1 epilogue of one TMEM lane (= one row): columns [0, hcols) from taddr
+// hold a = x W1 and columns [b_off, b_off + hcols) hold b = x W3 for the same
+// output columns; h = SiLU(a) * b (silu_times).  hrow points at the row's
+// first output column x0.  With `tma` the warp's 32 rows go out through `map`
+// (bf16, 64-byte rows, 64-byte swizzle) at (x0 + c, y0).  ba / bb (nullable)
+// are the biases of output column x0 for a and b.
+__device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, uint32_t b_off, bool valid,
+                                                bool tma, __nv_bfloat16* hrow, int hcols,
                                                 const CUtensorMap* map, EpiStage& st, int x0,
                                                 int y0, int lane, const float* ba,
                                                 const float* bb) {
@@ -231,7 +232,7 @@ __device__ __forceinline__ void epilogue_swiglu(uint32_t taddr, bool valid, bool
     for (int c = 0; c < hcols; c += 32) {
         uint32_t ra[32], rb[32];
         tmem_ld_32cols(taddr + c, ra);
-        tmem_ld_32cols(taddr + hcols + c, rb);
+        tmem_ld_32cols(taddr + b_off + c, rb);
         tmem_ld_wait();
         if (ba) add_bias_32(ra, ba + c);
         if (bb) add_bias_32(rb, bb + c);
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* ba = p.bias_a ? p.bias_a + boff : nullptr;
             const float* bb = p.bias_b ? p.bias_b + boff : nullptr;
             if (kSwiGLU)
-                epilogue_swiglu(taddr, valid, tma,
+                epilogue_swiglu(taddr, (uint32_t)p.n_tile_out, valid, tma,
                                 reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + ti.n0,
                                 p.n_tile_out, &tmOut, st, ti.n0, y0, lane, ba, bb);
             else
@@ -528,13 +529,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel
-// Same roles and tile enumeration, but a cluster of two CTAs on two SMs works on
-// a 256-row tile with one tcgen05 MMA of M = 256 (cta_group::2): CTA rank r
-// holds A rows [128r, 128r+128) of the tile and half of the B columns (GEMM1:
-// rank 0 the W1 columns, rank 1 the W3 columns; GEMM2: column halves of W2),
-// and receives its own 128 rows of D in its TMEM.  Per CTA a stage is 32 KB
-// (A 16 KB + half of B 16 KB) instead of 48 KB, so six stages fit, and each
-// SM reads half as many B bytes per MMA.
+// Same roles, but a cluster of two CTAs on two SMs shares each tile's MMAs
+// (tcgen05.mma.cta_group::2): CTA rank r holds its share of the A rows and half
+// of the B columns, and receives its own rows of D in its TMEM.  Per CTA a
+// stage is 32 KB (A 16 KB + half of B 16 KB), so six stages fit, and each SM
+// reads half as many B bytes per MMA as a single CTA with the same tile.
+//
+// Tile kinds.  An expert's rows are cut into "full" tiles of 256 rows (M = 256:
+// 128 rows per CTA; the last one may be ragged) and, when the last remainder
+// is at most 128 rows, one "half" tile of 128 rows (M = 128: 64 rows per CTA,
+// loaded through a 64-row A box), which does half a full tile's MMA work
+// instead of padding the remainder to 256 rows.
+//
+// TMEM layout of one accumulator (256 columns) in each CTA:
+//   full tile: lane l = row l of the CTA's 128 rows, column c = MMA column c;
+//   half tile: lane l = row l % 64 of the CTA's 64 rows, MMA columns
+//              128 (l / 64) + c in columns c < 128.
+// B columns: GEMM2 (N = 256 output columns) -- CTA r holds output columns
+// [128 r, 128 r + 128) of the tile.  GEMM1 (128 h columns per tile) -- CTA r
+// holds W1 columns [64 r, 64 r + 64) and then the same W3 columns, so MMA
+// column order is a(0..63) b(0..63) a(64..127) b(64..127): in both tile kinds
+// every lane holds a and b of the same h columns, 64 columns apart.
+//
+// Dealing (identical in every role and both CTAs): all tiles round-robin over
+// the P pairs, full tiles first, then half tiles (see deal_pair_tile).
 //
 // Synchronisation: both CTAs' TMA loads count their bytes on the leader's
 // (rank 0) full barrier, which only the leader arms with the bytes of both;
@@ -544,16 +562,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 // barrier (count 8).  Cluster barriers at start (barrier initialisation) and
 // end (before the pair frees its tensor memory) are reached by every thread of
 // both CTAs unconditionally; every mbarrier wait in between is bounded.
-constexpr int kPM = 256;                                       // rows per pair tile
+constexpr int kPM = 256;                                       // rows per full pair tile
+constexpr int kPHalf = 128;                                    // rows per half pair tile
 constexpr int kPairStages = 6;
-constexpr int kPairBBoxes = 2;                                 // B boxes per CTA per stage (max)
+constexpr int kPairBBoxes = 2;                                 // B boxes per CTA per stage
 constexpr int kPairStageBytes = kABytes + kPairBBoxes * kBBoxBytes;   // 32 KB
 constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + kEpiBytes + 1024;
 constexpr int kPairMinRows = 512;
+constexpr int kPairMinRounds = 8;
+
+// Tile of the pair enumeration: ids [0, F) are full tiles (expert-major, in
+// the rasterisation groups of decode_tile_rows over `s_full`), ids [F, F + H)
+// half tiles (expert-major, n fastest).
+struct PairTile {
+    TileInfo ti;
+    bool half;
+};
+
+__device__ __forceinline__ PairTile decode_pair_tile(int id, int F, const int* s_full,
+                                                     const int* s_half, const int* off,
+                                                     int n_tiles, int n_tile_out, int group_m) {
+    PairTile pt;
+    if (id < F) {
+        pt.ti = decode_tile_rows(id, s_full, off, n_tiles, n_tile_out, kPM, group_m);
+        pt.half = false;
+    } else {
+        const int j = id - F;
+        const int hm = j / n_tiles;
+        int e = 0;
+        while (hm >= s_half[e + 1]) ++e;
+        pt.ti.e = e;
+        pt.ti.row0 = off[e] + (s_full[e + 1] - s_full[e]) * kPM;
+        pt.ti.rows = off[e + 1] - pt.ti.row0;
+        pt.ti.n0 = (j - hm * n_tiles) * n_tile_out;
+        pt.half = true;
+    }
+    return pt;
+}
+
+// The i-th tile (id) dealt to pair p of P, or -1 past its last: the tiles go
+// round-robin in enumeration order, full tiles first, then half tiles.  A half
+// tile has half the MMA work of a full one but the same B bytes per stage, so
+// it takes about 0.7 of a full tile's time; dealing the half tiles after all
+// full tiles hands them to the pairs with one full tile fewer first, and no
+// pair runs two half tiles where a full tile would have done.
+__device__ __forceinline__ int deal_pair_tile(int i, int p, int P, int F, int H) {
+    const int id = p + i * P;
+    return id < F + H ? id : -1;
+}
 
 template <bool kSwiGLU>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmA64,
                             const __grid_constant__ CUtensorMap tmB0,
                             const __grid_constant__ CUtensorMap tmB1,
                             const __grid_constant__ CUtensorMap tmOut, const Params p) {
@@ -568,7 +629,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __shared__ uint64_t drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int s_off[kMaxE + 1];
-    __shared__ int s_mt[kMaxE + 1];
+    __shared__ int s_full[kMaxE + 1];
+    __shared__ int s_half[kMaxE + 1];
     __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5;
@@ -593,6 +655,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmA64);
         tma_prefetch_map(&tmB0);
         if (kSwiGLU) tma_prefetch_map(&tmB1);
         tma_prefetch_map(&tmOut);
@@ -603,13 +666,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     grid_dependency_wait();
     if (threadIdx.x == 0) {
-        int acc = 0;
-        s_mt[0] = 0;
+        // full m-tiles (256 rows; a remainder above 128 rows is a ragged full
+        // tile) and half m-tiles (a remainder of 1..128 rows) per expert
+        int nf = 0, nh = 0;
+        s_full[0] = 0;
+        s_half[0] = 0;
         for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
         for (int e = 0; e < p.E; ++e) {
             const int cnt = max(0, s_off[e + 1] - s_off[e]);
-            acc += (cnt + kPM - 1) / kPM;
-            s_mt[e + 1] = acc;
+            const int rem = cnt % kPM;
+            nf += cnt / kPM + (rem > kPHalf ? 1 : 0);
+            nh += (rem > 0 && rem <= kPHalf) ? 1 : 0;
+            s_full[e + 1] = nf;
+            s_half[e + 1] = nh;
         }
     }
     tc_fence_before_sync();
@@ -619,10 +688,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = tmem_slot;
 
     const int n_tiles = p.n_out / p.n_tile_out;
-    const int total_tiles = s_mt[p.E] * n_tiles;
+    const int F = s_full[p.E] * n_tiles;
+    const int H = s_half[p.E] * n_tiles;
     const int kb_count = p.K / kBK;
     const int boxes = p.n_boxes;  // B boxes per CTA per stage
-    const TileDeal deal = deal_tiles(pair, npairs, total_tiles);  // same for both CTAs
 
     if (warp == 0) {
         if (lane == 0) {
@@ -632,12 +701,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t issued_mask = 0, issued_parity = 0;
             int issued = 0;
             bool ok = true;
-            const uint32_t tx_pair = 2u * (kABytes + boxes * kBBoxBytes);
             const uint32_t leader_full0 = map_to_cta(smem_u32(&full_bar[0]), 0);
-            for (int t = deal.first; t < total_tiles && ok; t += deal.stride) {
-                const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM, p.group_m);
-                const int my_row0 = ti.row0 + (int)rank * kBM;
-                const int wrow0 = ti.e * p.K;
+            for (int i = 0; ok; ++i) {
+                const int id = deal_pair_tile(i, pair, npairs, F, H);
+                if (id < 0) break;
+                const PairTile pt = decode_pair_tile(id, F, s_full, s_half, s_off, n_tiles,
+                                                     p.n_tile_out, p.group_m);
+                const CUtensorMap* am = pt.half ? &tmA64 : &tmA;
+                const int my_row0 = pt.ti.row0 + (int)rank * (pt.half ? kPHalf / 2 : kBM);
+                const uint32_t tx_pair =
+                    2u * ((pt.half ? kABytes / 2 : kABytes) + boxes * kBBoxBytes);
+                const int wrow0 = pt.ti.e * p.K;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (p.stall_after >= 0 && issued >= p.stall_after) {
                         ok = false;  // test hook: both producers stop at the same stage
@@ -654,13 +728,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx_pair);
                     const int wrow = wrow0 + kb * kBK;
                     if (kSwiGLU) {
-                        const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
-                        tma_load_3d_pair(sB, mb, bar, 0, wrow, ti.n0 / kBoxN);
+                        // 64 W1 columns and the same 64 W3 columns of this CTA's half
+                        const int chunk = (pt.ti.n0 + (int)rank * kBoxN) / kBoxN;
+                        tma_load_3d_pair(sB, &tmB0, bar, 0, wrow, chunk);
+                        tma_load_3d_pair(sB + kBBoxBytes, &tmB1, bar, 0, wrow, chunk);
                     } else {
-                        const int c0 = ti.n0 + (int)rank * boxes * kBoxN;
+                        const int c0 = pt.ti.n0 + (int)rank * boxes * kBoxN;
                         tma_load_3d_pair(sB, &tmB0, bar, 0, wrow, c0 / kBoxN);
                     }
-                    tma_load_2d_pair(sA, &tmA, bar, kb * kBK, my_row0);
+                    tma_load_2d_pair(sA, am, bar, kb * kBK, my_row0);
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     ++issued;
@@ -681,7 +757,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer (leader only)
-            const uint32_t idesc = idesc_bf16_f32(kPM, 2 * boxes * kBoxN, false, true);
+            const uint32_t idesc_full = idesc_bf16_f32(kPM, 2 * boxes * kBoxN, false, true);
+            const uint32_t idesc_half = idesc_bf16_f32(kPHalf, 2 * boxes * kBoxN, false, true);
             const uint64_t adesc0 = desc_kmajor_sw128(smem_u32(smem));
             const uint64_t bdesc0 = desc_mnmajor_sw128(smem_u32(smem) + kABytes, kBBoxBytes);
             int stage = 0;
@@ -689,7 +766,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = deal.first; t < total_tiles && ok; t += deal.stride) {
+            for (int i = 0; ok; ++i) {
+                const int id = deal_pair_tile(i, pair, npairs, F, H);
+                if (id < 0) break;
+                const uint32_t idesc = id >= F ? idesc_half : idesc_full;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns) || s_abort) {
                     record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                     ok = false;
@@ -732,13 +812,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
-        const int row_in_cta = q * 32 + lane;
         EpiStage st{smem + kPairStages * kPairStageBytes + q * kEpiWarpBytes, 0u};
         int acc = 0;
         uint32_t acc_phase = 0;
         const uint32_t leader_acc_empty0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
-        for (int t = deal.first; t < total_tiles; t += deal.stride) {
-            const TileInfo ti = decode_tile_rows(t, s_mt, s_off, n_tiles, p.n_tile_out, kPM, p.group_m);
+        for (int i = 0;; ++i) {
+            const int id = deal_pair_tile(i, pair, npairs, F, H);
+            if (id < 0) break;
+            const PairTile pt = decode_pair_tile(id, F, s_full, s_half, s_off, n_tiles,
+                                                 p.n_tile_out, p.group_m);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
                 if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
@@ -747,23 +829,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const uint32_t taddr = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
-            const int row_in_tile = (int)rank * kBM + row_in_cta;
-            const bool valid = row_in_tile < ti.rows;
-            const int warp_row0 = (int)rank * kBM + q * 32;
-            const bool tma = warp_row0 + 32 <= ti.rows;  // warp-uniform
-            const int64_t grow = (int64_t)ti.row0 + row_in_tile;
-            const int y0 = ti.row0 + warp_row0;
-            const int64_t boff = (int64_t)ti.e * p.n_out + ti.n0;
-            const float* ba = p.bias_a ? p.bias_a + boff : nullptr;
-            const float* bb = p.bias_b ? p.bias_b + boff : nullptr;
-            if (kSwiGLU)
-                epilogue_swiglu(taddr, valid, tma,
-                                reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + ti.n0,
-                                p.n_tile_out, &tmOut, st, ti.n0, y0, lane, ba, bb);
-            else
+            // this warp's rows of the tile and the MMA columns its lanes hold
+            const int warp_row0 = pt.half ? (int)rank * (kPHalf / 2) + (q & 1) * 32
+                                          : (int)rank * kBM + q * 32;
+            const int col_half = pt.half ? (q >> 1) : 0;  // half tile: which 128 MMA columns
+            const int row_in_tile = warp_row0 + lane;
+            const bool valid = row_in_tile < pt.ti.rows;
+            const bool tma = warp_row0 + 32 <= pt.ti.rows;  // warp-uniform
+            const int64_t grow = (int64_t)pt.ti.row0 + row_in_tile;
+            const int y0 = pt.ti.row0 + warp_row0;
+            const int64_t boff = (int64_t)pt.ti.e * p.n_out;
+            if (kSwiGLU) {
+                // h columns [x0, x0 + 64): a in TMEM columns [c0, c0 + 64), b 64 further
+                for (int seg = 0; seg < (pt.half ? 1 : 2); ++seg) {
+                    const int part = pt.half ? col_half : seg;
+                    const int x0 = pt.ti.n0 + part * 64;
+                    epilogue_swiglu(taddr + (uint32_t)((pt.half ? 0 : part) * 128), 64u, valid,
+                                    tma,
+                                    reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.n_out + x0,
+                                    64, &tmOut, st, x0, y0, lane,
+                                    p.bias_a ? p.bias_a + boff + x0 : nullptr,
+                                    p.bias_b ? p.bias_b + boff + x0 : nullptr);
+                }
+            } else {
+                const int ncols = pt.half ? boxes * kBoxN : 2 * boxes * kBoxN;
+                const int x0 = pt.ti.n0 + col_half * boxes * kBoxN;
                 epilogue_store_f32(taddr, valid, tma,
-                                   reinterpret_cast<float*>(p.out) + grow * p.n_out + ti.n0,
-                                   2 * boxes * kBoxN, &tmOut, st, ti.n0, y0, lane, ba);
+                                   reinterpret_cast<float*>(p.out) + grow * p.n_out + x0, ncols,
+                                   &tmOut, st, x0, y0, lane,
+                                   p.bias_a ? p.bias_a + boff + x0 : nullptr);
+            }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * (uint32_t)sizeof(uint64_t));
@@ -920,14 +1015,14 @@ static int max_pairs() {
 }
 
 template <bool kSwiGLU>
-static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                       const CUtensorMap& out, const Params& p, int max_tiles,
-                       cudaStream_t stream) {
+static int launch_pair(const CUtensorMap& a, const CUtensorMap& a64, const CUtensorMap& b0,
+                       const CUtensorMap& b1, const CUtensorMap& out, const Params& p,
+                       int max_tiles, cudaStream_t stream) {
     const int pairs = max_pairs<kSwiGLU>();  // also sets the shared-memory attribute
     if (pairs <= 0) return MOE_ERR_CUDA;
     const int grid = 2 * max(1, min(pairs, max_tiles));
     return launch_pdl(expert_gemm_pair_kernel<kSwiGLU>, dim3(grid), dim3(kThreads),
-                      kPairSmemBytes, stream, a, b0, b1, out, p) == cudaSuccess
+                      kPairSmemBytes, stream, a, a64, b0, b1, out, p) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }
@@ -941,25 +1036,36 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     using namespace gemm;
     const int R = s.T * s.k;
     if (R == 0) return MOE_OK;
-    CUtensorMap mx, mh, m1, m3, m2, oh, oo;
+    CUtensorMap mx, mh, mx64, mh64, m1, m3, m2, oh, oo;
     if (!make_map(&mx, x_sorted, (uint64_t)R, (uint64_t)s.d, kBM) ||
         !make_map(&mh, h, (uint64_t)R, (uint64_t)s.d_ff, kBM) ||
+        !make_map(&mx64, x_sorted, (uint64_t)R, (uint64_t)s.d, kPHalf / 2) ||
+        !make_map(&mh64, h, (uint64_t)R, (uint64_t)s.d_ff, kPHalf / 2) ||
         !make_out_map(&oh, h, (uint64_t)R, (uint64_t)s.d_ff, false) ||
         !make_out_map(&oo, o, (uint64_t)R, (uint64_t)s.d, true))
         return MOE_ERR_CUDA;
-    // GEMM2 (long K = d_ff) runs on CTA pairs (256-row tiles, M = 256 MMAs) once
-    // there are at least kPairMinRows routed rows; GEMM1 (K = d, SwiGLU epilogue)
-    // stays on single CTAs with 128-row tiles, whose smaller padding of ragged
-    // expert groups outweighs the pair's saving (measured on the Mixtral shapes),
-    // and so does decode-sized work for both.
-    const bool pairs1 = false;
+    // The down projection runs on CTA pairs (256-row full tiles, 128-row half
+    // tiles for remainders of at most 128 rows) once there are at least
+    // kPairMinRows routed rows.  GEMM1 does when its pair tiles fill at least
+    // kPairMinRounds rounds of the pairs: with fewer, the single CTA's 128-row
+    // tiles quantise better (measured: the quarter-width batch, R = 2048, three
+    // pair rounds, ran 4 % slower on pairs; the Mixtral prefill batch, 48
+    // rounds, 8 % faster).  Decode-sized work runs on single CTAs, where every
+    // tile streams its own weight slice.
     const bool pairs2 = R >= kPairMinRows;
-    auto mtiles = [&](int tile_rows) { return (R + tile_rows - 1) / tile_rows + s.E; };
+    const int64_t pair_tiles1 = ((int64_t)R / kPM) * (s.d_ff / 128);
+    const bool pairs1 = pairs2 && pair_tiles1 >= (int64_t)kPairMinRounds * max_pairs<true>();
+    // upper bound on the number of tiles of either kind
+    auto mtiles = [&](int tile_rows) { return (R + tile_rows - 1) / tile_rows + 2 * s.E; };
     // m-tiles per rasterisation group: as many as keep the group's activation
-    // rows (tile_rows x K bf16 each) within ~48 MB of the 126 MB L2.
+    // rows (tile_rows x K bf16 each) within 16 MB.  The 126 MB L2 is split over
+    // the two dies, and the weight slices of the column tiles in flight stream
+    // through it too; on the skewed batch (experts of up to 33 pair m-tiles)
+    // 16 MB groups ran the expert GEMMs 2.5 % faster than 48 MB groups, and the
+    // prefill batch's experts (4 m-tiles) fit either way.
     auto group_rows = [](int tile_rows, int K) {
         const int64_t per_tile = (int64_t)tile_rows * K * 2;
-        return (int)std::max<int64_t>(1, (int64_t(48) << 20) / per_tile);
+        return (int)std::max<int64_t>(1, (int64_t(16) << 20) / per_tile);
     };
 
     Params p1{};
@@ -970,24 +1076,23 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.E = s.E;
     p1.K = s.d;
     p1.n_out = s.d_ff;
-    // GEMM1 tiles cover 128 h columns: 2 weight boxes of W1 and 2 of W3 on one
-    // CTA (or one matrix per CTA of a pair).  Narrower 64-column tiles, which
-    // balance small batches across the SMs better, were measured slower at
-    // decode: every tile also streams a full 128-row A tile.
+    // GEMM1 tiles cover 128 h columns: on one CTA 2 weight boxes of W1 and 2 of
+    // W3; on a pair each CTA 1 box of W1 and the same columns of W3.  Narrower
+    // 64-column tiles, which balance small batches across the SMs better, were
+    // measured slower at decode: every tile also streams a full 128-row A tile.
     p1.n_tile_out = 128;
     p1.n_boxes = pairs1 ? 2 : 4;  // per CTA
     p1.stall_after = stall_after;
     p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
     p1.bias_a = b1;
     p1.bias_b = b3;
-    // weight boxes: W1 / W3 chunks per copy = half of the CTA's B boxes (single
-    // CTA: both matrices) or all of them (pair: one matrix per CTA)
-    const uint32_t ch1 = pairs1 ? (uint32_t)p1.n_boxes : (uint32_t)p1.n_boxes / 2;
+    // weight boxes: W1 / W3 chunks per copy = half of the CTA's B boxes
+    const uint32_t ch1 = (uint32_t)p1.n_boxes / 2;
     if (!make_weight_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1) ||
         !make_weight_map(&m3, W3, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1))
         return MOE_ERR_CUDA;
     const int t1 = mtiles(pairs1 ? kPM : kBM) * (s.d_ff / p1.n_tile_out);
-    int rc = pairs1 ? launch_pair<true>(mx, m1, m3, oh, p1, t1, stream)
+    int rc = pairs1 ? launch_pair<true>(mx, mx64, m1, m3, oh, p1, t1, stream)
                     : launch<true>(mx, m1, m3, oh, p1, t1, stream);
     if (rc != MOE_OK) return rc;
     if (mid_event && cudaEventRecord(static_cast<cudaEvent_t>(mid_event), stream) != cudaSuccess)
@@ -1006,7 +1111,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     if (!make_weight_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, (uint32_t)p2.n_boxes))
         return MOE_ERR_CUDA;
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
-    return pairs2 ? launch_pair<false>(mh, m2, m2, oo, p2, t2, stream)
+    return pairs2 ? launch_pair<false>(mh, mh64, m2, m2, oo, p2, t2, stream)
                   : launch<false>(mh, m2, m2, oo, p2, t2, stream);
 }
 

@@ -6,15 +6,31 @@
 //
 // The contraction x[T,d] . Wg[d,E] is skinny (E = 8) and HBM-bound on reading
 // x once; it runs on mma.sync m16n8k16 (bf16 in, fp32 accumulate) so the issue
-// slots stay free for loads.  A warp owns 16 tokens and 1/KSPLIT of d; the
-// KSPLIT partial sums are added in a fixed order, so results are deterministic.
-// KSPLIT grows when there are few tokens (decode) so that more warps share the
-// one tile of 16 tokens and the kernel is not bound by one warp's load latency.
+// slots stay free for loads.
 //
-// k-permutation: a dot product may pair its terms in any order, so a lane loads
+// Work split.  A warp owns one tile of 16 tokens and a contiguous range of the
+// 32-wide k blocks of d.  The d axis is cut into KS = 8 C ranges: the 8 warps of
+// a CTA take 8 of them, and a cluster of C CTAs (C = 1, 2, 4 or 8) covers all
+// of d for the same token tile.  C grows when there are few token tiles
+// (decode: one tile over 8 CTAs) so that the loads spread over more SMs; each
+// CTA stages only the W_r rows of its own k range.  The KS partial sums of a
+// logit are added in range order by one warp of the cluster's first CTA, which
+// reads the other CTAs' partials through distributed shared memory; the order
+// depends only on C and d, so results are deterministic and a caller that runs
+// one batch in token chunks can pass the whole batch's C.
+//
+// W_r staging.  W_r's rows (8 experts = 16 bytes per row and 8-expert plane)
+// are copied as they are, with 16-byte asynchronous copies, into shared memory,
+// row r of a 32-row k block at 16-byte slot r ^ (((r >> 3) & 3) << 1): the copy
+// needs no registers and overlaps the first x loads.  B fragments come out of
+// it with ldmatrix .trans, whose per-lane row addresses pick the rows in the
+// order of the k permutation below; the slot swizzle makes the eight rows of
+// every 8x8 matrix fall in distinct bank groups.
+//
+// k permutation: a dot product may pair its terms in any order, so a lane loads
 // 8 consecutive x elements (one 16-byte load) and feeds them to two MMAs as
-// fragment positions {2t,2t+1,2t+8,2t+9}; the router weights are staged in
-// shared memory in the matching order (one 16-byte load per lane per 32 k).
+// fragment positions {2t,2t+1,2t+8,2t+9}; the B fragments are read in the same
+// order (matrix m of a k block holds rows 8i + 2m + {0,1}, i = 0..3).
 //
 // Top-k: the four lanes of a quad hold the E logits of one token; k rounds of a
 // quad-shuffle argmax pick the largest logit not yet taken, lower expert index
@@ -28,13 +44,16 @@
 
 #include "common.cuh"
 #include "router.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace router {
 
-constexpr int kWarps = 16;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxK = 8;
+constexpr int kMaxCluster = 8;
+constexpr int kGroup = 8;  // k blocks whose x loads are issued together
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
@@ -46,234 +65,310 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&b)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// 16-byte slot of row r (local to the CTA's staged range) of a W_r plane.
+__device__ __forceinline__ int w_slot(int r) { return r ^ (((r >> 3) & 3) << 1); }
+
 __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
     return v > bv || (v == bv && id < bid) || bid == INT_MAX;
 }
 
-template <int NT, int KSPLIT>
-__global__ void __launch_bounds__(kThreads, 1)
-    router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
-                  const float* __restrict__ bias, int T, int d, int E, int k,
-                  int32_t* __restrict__ idx, float* __restrict__ gate,
-                  float* __restrict__ logits) {
-    constexpr int kSlots = kWarps / KSPLIT;  // token tiles of 16 per block iteration
-    extern __shared__ uint4 s_wg[];  // [d/32][NT][32 lanes] x 8 bf16
-    __shared__ float s_red[kSlots][KSPLIT][NT][32][4];
-    grid_dependency_wait();
-
-    // Stage W_r in fragment order: entry (kb, nt, lane) holds
-    // Wg[kb*32 + (lane&3)*8 + j][nt*8 + (lane>>2)] for j = 0..7 (zero for n >= E),
-    // i.e. element (r, n) goes to half-word r % 8 of entry
-    // (r / 32, n / 8, (n % 8) * 4 + (r % 32) / 8).  Each thread reads whole rows
-    // of W_r (16-byte loads when a row is a multiple of 16 bytes) and scatters
-    // their elements; a warp's 32 consecutive rows land in one 64-byte span per
-    // column, so the 2-byte shared stores do not conflict.
-    uint16_t* s_half = reinterpret_cast<uint16_t*>(s_wg);
-    auto put = [&](int r, int n, uint16_t v) {
-        const int entry = ((r >> 5) * NT + (n >> 3)) * 32 + (n & 7) * 4 + ((r & 31) >> 3);
-        s_half[entry * 8 + (r & 7)] = v;
-    };
-    if ((E & 7) == 0) {
-        const int vec = E >> 3;  // 16-byte pieces per row
-#pragma unroll 4
-        for (int r = threadIdx.x; r < d; r += blockDim.x) {
-            const uint4* row = reinterpret_cast<const uint4*>(wg + (int64_t)r * E);
-            for (int q = 0; q < vec; ++q) {
-                const uint4 v = __ldg(row + q);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Top-k of the logits v (fragment layout of the MMA accumulator: v[nt][i] is
+// token (i < 2 ? g : g + 8) of the tile, expert nt*8 + 2*t4 + (i & 1)), softmax
+// over the k, and the stores of idx, gate and (optionally) the logits.  Kept out
+// of line: it runs in one warp per tile, after the x loads' registers are dead.
+template <int NT>
+__device__ __noinline__ void select_and_store(float (&v)[NT][4], int tile, int T, int E, int k,
+                                              int g, int t4, int32_t* __restrict__ idx,
+                                              float* __restrict__ gate,
+                                              float* __restrict__ logits) {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    put(r, q * 8 + 2 * h, (uint16_t)(w[h] & 0xFFFFu));
-                    put(r, q * 8 + 2 * h + 1, (uint16_t)(w[h] >> 16));
+    for (int half = 0; half < 2; ++half) {
+        const int row = tile * 16 + g + 8 * half;
+        const bool rv = row < T;
+        if (logits && rv) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int n = nt * 8 + 2 * t4 + j;
+                    if (n < E) logits[(int64_t)row * E + n] = v[nt][2 * half + j];
+                }
+        }
+        uint32_t taken = 0;  // bit (nt*2 + j) of this lane's candidates
+        float sel_v[kMaxK];
+        int sel_id[kMaxK];
+#pragma unroll
+        for (int s = 0; s < kMaxK; ++s) {
+            if (s >= k) break;
+            float bv = -FLT_MAX;
+            int bid = INT_MAX;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int n = nt * 8 + 2 * t4 + j;
+                    const int bit = nt * 2 + j;
+                    const float cv = v[nt][2 * half + j];
+                    if (n < E && !(taken & (1u << bit)) && better(cv, n, bv, bid)) {
+                        bv = cv;
+                        bid = n;
+                    }
+                }
+#pragma unroll
+            for (int off = 1; off <= 2; off <<= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+                if (oid != INT_MAX && better(ov, oid, bv, bid)) {
+                    bv = ov;
+                    bid = oid;
                 }
             }
+            // the lane that holds the winner marks it taken
+            if (bid != INT_MAX && ((bid & 7) >> 1) == t4) taken |= 1u << ((bid >> 3) * 2 + (bid & 1));
+            sel_v[s] = bv;
+            sel_id[s] = bid;
         }
-    } else {
-        for (int r = threadIdx.x; r < d; r += blockDim.x)
-            for (int n = 0; n < NT * 8; ++n)
-                put(r, n, n < E ? __ldg(wg + (int64_t)r * E + n) : (uint16_t)0);
+        if (rv && t4 == 0) {
+            const float m = sel_v[0];
+            float den = 0.f;
+            float ex[kMaxK];
+#pragma unroll
+            for (int s = 0; s < kMaxK; ++s) {
+                if (s >= k) break;
+                ex[s] = expf(sel_v[s] - m);
+                den = __fadd_rn(den, ex[s]);
+            }
+#pragma unroll
+            for (int s = 0; s < kMaxK; ++s) {
+                if (s >= k) break;
+                idx[(int64_t)row * k + s] = sel_id[s];
+                gate[(int64_t)row * k + s] = __fdiv_rn(ex[s], den);
+            }
+        }
     }
-    __syncthreads();
+}
 
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int slot = warp / KSPLIT;
-    const int kq = warp % KSPLIT;
+// Dynamic shared memory: NT planes of W_r rows [rows_cap][16 bytes], then the
+// partial sums [2 buffers][kWarps][32 lanes][NT] float4.
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 2)
+    router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
+                  const float* __restrict__ bias, int T, int d, int E, int k, int C,
+                  int32_t* __restrict__ idx, float* __restrict__ gate,
+                  float* __restrict__ logits) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
     const int g = lane >> 2;
     const int t4 = lane & 3;
-    const int kper = d / KSPLIT;
-    const int ntiles = (T + 15) / 16;
+    const int rank = (int)sm100::cluster_ctarank();
+    const int nkb = d >> 5;
+    const int KS = C * kWarps;
+    const int rows_cap = ((nkb + C - 1) / C) * 32;
+    const int cta_kb0 = (rank * nkb) / C;
+    const int cta_rows = ((((rank + 1) * nkb) / C) - cta_kb0) * 32;
+    const uint32_t s_w = sm100::smem_u32(smem);
+    const uint32_t s_part = s_w + (uint32_t)(NT * rows_cap * 16);
+    grid_dependency_wait();
 
-    for (int base = blockIdx.x * kSlots; base < ntiles; base += gridDim.x * kSlots) {
-        const int tile = base + slot;
+    // Stage this CTA's rows of W_r, plane by plane (8 experts per plane).
+    if ((E & 7) == 0) {
+        for (int i = tid; i < NT * cta_rows; i += kThreads) {
+            const int nt = i / cta_rows;
+            const int r = i - nt * cta_rows;
+            cp_async_16(s_w + (uint32_t)((nt * rows_cap + w_slot(r)) * 16),
+                        wg + (int64_t)(cta_kb0 * 32 + r) * E + nt * 8);
+        }
+    } else {
+        for (int i = tid; i < NT * cta_rows * 8; i += kThreads) {
+            const int j = i & 7;
+            const int rest = i >> 3;
+            const int nt = rest / cta_rows;
+            const int r = rest - nt * cta_rows;
+            const int n = nt * 8 + j;
+            const uint16_t v = n < E ? wg[(int64_t)(cta_kb0 * 32 + r) * E + n] : (uint16_t)0;
+            reinterpret_cast<uint16_t*>(smem)[(nt * rows_cap + w_slot(r)) * 8 + j] = v;
+        }
+    }
+
+    const int q = rank * kWarps + warp;          // this warp's k range
+    const int kb_lo = (q * nkb) / KS;
+    const int kb_hi = ((q + 1) * nkb) / KS;
+    // ldmatrix: lane supplies row i = lane & 7 of matrix m = lane >> 3, i.e. row
+    // 8 (i >> 1) + 2 m + (i & 1) of the k block
+    const int lrow = 8 * ((lane & 7) >> 1) + 2 * (lane >> 3) + (lane & 1);
+    const uint32_t lane_off = (uint32_t)(w_slot(lrow) * 16);
+    const int ntiles = (T + 15) >> 4;
+    const int cluster = blockIdx.x / C;
+    const int nclusters = gridDim.x / C;
+
+    int it = 0;
+    for (int tile = cluster; tile < ntiles; tile += nclusters, ++it) {
         float c[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
-        if (tile < ntiles) {
-            const int r0 = tile * 16 + g;
-            const int r1 = r0 + 8;
-            const bool v0 = r0 < T, v1 = r1 < T;
-            const uint4* x0 = reinterpret_cast<const uint4*>(x + (int64_t)(v0 ? r0 : 0) * d);
-            const uint4* x1 = reinterpret_cast<const uint4*>(x + (int64_t)(v1 ? r1 : 0) * d);
-            const int kbeg = kq * kper, kend = kbeg + kper;
-#pragma unroll 4
-            for (int kb = kbeg; kb < kend; kb += 32) {
-                const int ci = (kb >> 3) + t4;
-                const uint4 a0 = v0 ? __ldg(x0 + ci) : make_uint4(0, 0, 0, 0);
-                const uint4 a1 = v1 ? __ldg(x1 + ci) : make_uint4(0, 0, 0, 0);
+        const int r0 = tile * 16 + g;
+        const int r1 = r0 + 8;
+        const bool v0 = r0 < T, v1 = r1 < T;
+        const uint4* x0 = reinterpret_cast<const uint4*>(x + (int64_t)(v0 ? r0 : 0) * d) + t4;
+        const uint4* x1 = reinterpret_cast<const uint4*>(x + (int64_t)(v1 ? r1 : 0) * d) + t4;
+        for (int kb = kb_lo, first = 1; first || kb < kb_hi; kb += kGroup, first = 0) {
+            const int n = min(kGroup, kb_hi - kb);
+            uint4 a0[kGroup], a1[kGroup];
+#pragma unroll
+            for (int j = 0; j < kGroup; ++j) {
+                if (j < n) {
+                    a0[j] = v0 ? __ldg(x0 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
+                    a1[j] = v1 ? __ldg(x1 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
+                }
+            }
+            if (first && it == 0) {  // W_r must have landed (every warp passes here once)
+                cp_async_wait_all();
+                __syncthreads();
+            }
+#pragma unroll
+            for (int j = 0; j < kGroup; ++j) {
+                if (j < n) {
+                    const uint32_t blk = s_w + (uint32_t)((kb + j - cta_kb0) * 32 * 16) + lane_off;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        uint32_t b[4];
+                        ldmatrix_x4_trans(blk + (uint32_t)(nt * rows_cap * 16), b);
+                        mma_bf16_16816(c[nt], a0[j].x, a1[j].x, a0[j].y, a1[j].y, b[0], b[1]);
+                        mma_bf16_16816(c[nt], a0[j].z, a1[j].z, a0[j].w, a1[j].w, b[2], b[3]);
+                    }
+                }
+            }
+        }
+        // partial sums of this warp, then one cluster barrier per tile (the buffer
+        // alternates: the reducing warp has read a buffer before it arrives at
+        // the barrier after next, which every writer of that buffer waits for)
+        float4* mine = reinterpret_cast<float4*>(smem + NT * rows_cap * 16) +
+                       (((it & 1) * kWarps + warp) * 32 + lane) * NT;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mine[nt] = make_float4(c[nt][0], c[nt][1], c[nt][2], c[nt][3]);
+        sm100::cluster_sync_all();
+        if (rank == 0 && warp == 0) {
+            float v[NT][4];
+            const uint32_t buf = s_part + (uint32_t)(((it & 1) * kWarps * 32 + lane) * NT * 16);
+            for (int qq = 0; qq < KS; ++qq) {
+                const uint32_t local = buf + (uint32_t)((qq % kWarps) * 32 * NT * 16);
+                const uint32_t src = sm100::map_to_cta(local, (uint32_t)(qq / kWarps));
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint4 b = s_wg[((kb >> 5) * NT + nt) * 32 + lane];
-                    mma_bf16_16816(c[nt], a0.x, a1.x, a0.y, a1.y, b.x, b.y);
-                    mma_bf16_16816(c[nt], a0.z, a1.z, a0.w, a1.w, b.z, b.w);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) s_red[slot][kq][nt][lane][i] = c[nt][i];
-        }
-        __syncthreads();
-        if (kq == 0 && tile < ntiles) {
-            // v[nt][i]: token (i < 2 ? g : g+8), expert nt*8 + 2*t4 + (i & 1)
-            float v[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float sum = s_red[slot][0][nt][lane][i];
-#pragma unroll
-                    for (int q = 1; q < KSPLIT; ++q) sum = __fadd_rn(sum, s_red[slot][q][nt][lane][i]);
-                    const int n = nt * 8 + 2 * t4 + (i & 1);
-                    if (bias && n < E) sum = __fadd_rn(sum, bias[n]);
-                    v[nt][i] = sum;
-                }
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int row = tile * 16 + g + 8 * half;
-                const bool rv = row < T;
-                if (logits && rv) {
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int n = nt * 8 + 2 * t4 + j;
-                            if (n < E) logits[(int64_t)row * E + n] = v[nt][2 * half + j];
-                        }
-                }
-                uint32_t taken = 0;  // bit (nt*2 + j) of this lane's candidates
-                float sel_v[kMaxK];
-                int sel_id[kMaxK];
-#pragma unroll
-                for (int s = 0; s < kMaxK; ++s) {
-                    if (s >= k) break;
-                    float bv = -FLT_MAX;
-                    int bid = INT_MAX;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int n = nt * 8 + 2 * t4 + j;
-                            const int bit = nt * 2 + j;
-                            const float cv = v[nt][2 * half + j];
-                            if (n < E && !(taken & (1u << bit)) && better(cv, n, bv, bid)) {
-                                bv = cv;
-                                bid = n;
-                            }
-                        }
-#pragma unroll
-                    for (int off = 1; off <= 2; off <<= 1) {
-                        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                        const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
-                        if (oid != INT_MAX && better(ov, oid, bv, bid)) {
-                            bv = ov;
-                            bid = oid;
-                        }
-                    }
-                    // the lane that holds the winner marks it taken
-                    if (bid != INT_MAX && ((bid & 7) >> 1) == t4)
-                        taken |= 1u << ((bid >> 3) * 2 + (bid & 1));
-                    sel_v[s] = bv;
-                    sel_id[s] = bid;
-                }
-                if (rv && t4 == 0) {
-                    const float m = sel_v[0];
-                    float den = 0.f;
-                    float ex[kMaxK];
-#pragma unroll
-                    for (int s = 0; s < kMaxK; ++s) {
-                        if (s >= k) break;
-                        ex[s] = expf(sel_v[s] - m);
-                        den = __fadd_rn(den, ex[s]);
-                    }
-#pragma unroll
-                    for (int s = 0; s < kMaxK; ++s) {
-                        if (s >= k) break;
-                        idx[(int64_t)row * k + s] = sel_id[s];
-                        gate[(int64_t)row * k + s] = __fdiv_rn(ex[s], den);
+                    const float4 p = ld_shared_cluster_f4(src + nt * 16);
+                    if (qq == 0) {
+                        v[nt][0] = p.x; v[nt][1] = p.y; v[nt][2] = p.z; v[nt][3] = p.w;
+                    } else {
+                        v[nt][0] = __fadd_rn(v[nt][0], p.x);
+                        v[nt][1] = __fadd_rn(v[nt][1], p.y);
+                        v[nt][2] = __fadd_rn(v[nt][2], p.z);
+                        v[nt][3] = __fadd_rn(v[nt][3], p.w);
                     }
                 }
             }
+            if (bias) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = nt * 8 + 2 * t4 + (i & 1);
+                        if (n < E) v[nt][i] = __fadd_rn(v[nt][i], bias[n]);
+                    }
+            }
+            select_and_store<NT>(v, tile, T, E, k, g, t4, idx, gate, logits);
         }
-        __syncthreads();
     }
+    cp_async_wait_all();
+    // no CTA leaves while the reducing warp may still read its partial sums
+    sm100::cluster_sync_all();
 }
 
 }  // namespace router
 
-int router_ksplit(const moe_shape& s) {
+int router_cluster(const moe_shape& s) {
     using namespace router;
     const int ntiles = (s.T + 15) / 16;
     const int sms = device_sm_count();
-    // Largest split of d (into 16, 8 or 4 parts, each a whole number of 32-wide
-    // k blocks) that still needs no more CTAs than there are SMs: few tokens
-    // (decode) then get 16 warps per tile instead of 4.
-    for (int cand : {16, 8}) {
-        const int ctas = (ntiles * cand + kWarps - 1) / kWarps;
-        if ((s.d / 32) % cand == 0 && ctas <= sms) return cand;
-    }
-    return 4;
+    const int nkb = s.d / 32;
+    // Largest cluster (1, 2, 4 or 8 CTAs per token tile) that keeps the grid
+    // within two CTAs per SM and gives every warp at least one k block.
+    int C = 1;
+    while (C < kMaxCluster && (int64_t)ntiles * (2 * C) <= 2 * sms && 2 * C * kWarps <= nkb) C *= 2;
+    return C;
 }
 
 int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
-                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int ksplit) {
+                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int cluster) {
     using namespace router;
     if (s.T == 0) return MOE_OK;
     const int NT = (s.E + 7) / 8;
-    const size_t smem = (size_t)s.d * NT * 16;
+    // The cluster size fixes the order in which the partial sums of a logit are
+    // added; a caller that runs one batch in token chunks passes the size chosen
+    // for the whole batch so every chunk rounds the same way.
+    const int C = cluster <= 0 ? router_cluster(s) : cluster;
+    if (C != 1 && C != 2 && C != 4 && C != 8) return MOE_ERR_INVALID_ARG;
+    const int nkb = s.d / 32;
+    const int rows_cap = ((nkb + C - 1) / C) * 32;
+    const size_t smem = (size_t)NT * rows_cap * 16 + (size_t)2 * kWarps * 32 * NT * 16;
     const int ntiles = (s.T + 15) / 16;
     const int sms = device_sm_count();
-    // The split decides the order in which the partial sums of a logit are
-    // added; a caller that runs one batch in token chunks passes the split of
-    // the whole batch so every chunk rounds the same way.
-    if (ksplit <= 0) ksplit = router_ksplit(s);
-    if (ksplit != 4 && ksplit != 8 && ksplit != 16) return MOE_ERR_INVALID_ARG;
-    if ((s.d / 32) % ksplit != 0) return MOE_ERR_INVALID_ARG;
-    const int slots = kWarps / ksplit;
-    const int grid = std::max(1, std::min(sms, (ntiles + slots - 1) / slots));
+    const int nclusters = std::max(1, std::min(ntiles, (2 * sms) / C));
     const uint16_t* xp = static_cast<const uint16_t*>(x);
     const uint16_t* wp = static_cast<const uint16_t*>(Wg);
     auto run = [&](auto kern) {
         if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem))
             return MOE_ERR_CUDA;
-        return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, xp, wp, bias, s.T, s.d,
-                          s.E, s.k, idx, gate, logits) == cudaSuccess
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(nclusters * C);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, kern, xp, wp, bias, s.T, s.d, s.E, s.k, C, idx, gate,
+                                  logits) == cudaSuccess
                    ? MOE_OK
                    : MOE_ERR_CUDA;
     };
-#define MOE_ROUTER_CASE(N)                                                  \
-    case N:                                                                 \
-        return ksplit == 16 ? run(router_kernel<N, 16>)                     \
-               : ksplit == 8 ? run(router_kernel<N, 8>) : run(router_kernel<N, 4>);
     switch (NT) {
-        MOE_ROUTER_CASE(1)
-        MOE_ROUTER_CASE(2)
-        MOE_ROUTER_CASE(3)
-        MOE_ROUTER_CASE(4)
-        default:
-            return MOE_ERR_UNSUPPORTED;
+        case 1: return run(router_kernel<1>);
+        case 2: return run(router_kernel<2>);
+        case 3: return run(router_kernel<3>);
+        case 4: return run(router_kernel<4>);
+        default: return MOE_ERR_UNSUPPORTED;
     }
-#undef MOE_ROUTER_CASE
 }
 
 }  // namespace moe

@@ -9,12 +9,13 @@
 namespace moe {
 
 // Logits (+ bias), top-k (ties -> lower expert id) and softmax over the k.
-// ksplit: how many parts d is split into for the partial sums of a logit (4, 8
-// or 16); 0 picks router_ksplit(s).
+// cluster: CTAs that share one token tile's contraction (1, 2, 4 or 8; d is
+// split into 8 * cluster ranges whose partial sums are added in order); 0 picks
+// router_cluster(s).
 int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
-                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int ksplit = 0);
+                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int cluster = 0);
 
-// The split launch_router picks for shape s (depends on T, d and the SM count).
-int router_ksplit(const moe_shape& s);
+// The cluster size launch_router picks for shape s (depends on T, d and the SM count).
+int router_cluster(const moe_shape& s);
 
 }  // namespace moe

@@ -260,7 +260,7 @@ def test_forward_deterministic_and_hostio_matches():
     assert torch.equal(y1.cpu(), y_host)
 
 
-@pytest.mark.parametrize("T", [2048, 4097], ids=["even-halves", "ragged-halves"])
+@pytest.mark.parametrize("T", [2048, 4097], ids=["2048-tokens", "4097-tokens"])
 def test_hostio_token_chunks_equal_the_whole_batch(T):
     """Large host-I/O batches run as a pipeline of token chunks; every row's
     arithmetic (including the router's summation split) is that of the whole
@@ -279,8 +279,8 @@ def test_hostio_token_chunks_equal_the_whole_batch(T):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
 
 
-@pytest.mark.parametrize("T,stall_chunk", [(2048, 0), (2048, 1), (300, 0)],
-                         ids=["first-of-two-chunks", "second-of-two-chunks", "one-chunk"])
+@pytest.mark.parametrize("T,stall_chunk", [(2048, 0), (2048, 1), (2048, 2), (300, 0)],
+                         ids=["first-of-three-chunks", "middle-chunk", "last-chunk", "one-chunk"])
 def test_hostio_reports_a_timeout_in_any_chunk(T, stall_chunk):
     """The host-I/O pipeline runs large batches as token chunks on one
     workspace; a wait that expires in an earlier chunk must not be cleared by a

@@ -57,3 +57,27 @@ def test_expert_rows_alone_match_the_batch(d_ff):
                       o[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64),
                       oracle.bf16_to_f64(xs_rows), row_expert, inp["W1"], inp["W3"], inp["W2"],
                       h_ref, o_ref)
+
+
+def test_rows_on_single_cta_tiles_match_the_cta_pair_batch():
+    """Experts of fewer than 512 rows alone run the down projection on single-CTA
+    128-row tiles; inside a batch of more than 512 rows they run on CTA pairs.
+    The bits must not change with the kernel that runs them."""
+    counts = [300, 130, 45, 400, 200, 1, 260, 90]
+    d, d_ff, E = 1024, 512, len(counts)
+    R = sum(counts)
+    assert R >= 512 and max(counts) < 512
+    inp = make_inputs(R, d, d_ff, E, 1, seed=85)
+    xs = inp["x"].cuda()
+    W1, W3, W2 = (inp[key].cuda() for key in ("W1", "W3", "W2"))
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    h, o, ws = moe.moe_expert_swiglu((R, d, d_ff, E, 1), xs, torch.from_numpy(off).cuda(),
+                                     W1, W3, W2)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    for e, c in enumerate(counts):
+        off_e = np.array([0] * (e + 1) + [c] * (E - e), dtype=np.int32)
+        h_e, o_e, ws_e = moe.moe_expert_swiglu((c, d, d_ff, E, 1), xs[off[e]:off[e + 1]].clone(),
+                                               torch.from_numpy(off_e).cuda(), W1, W3, W2)
+        assert moe.moe_read_device_status(ws_e) == moe.MOE_OK
+        assert torch.equal(h[off[e]:off[e + 1]], h_e), e
+        assert torch.equal(o[off[e]:off[e + 1]], o_e), e
