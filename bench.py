@@ -57,7 +57,8 @@ def parse(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the extras and the decode and skew objects of the prefill run")
+                    help="skip the extras and the decode, skew, quarter and tiny objects of the "
+                         "prefill run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--tokens", type=int, default=None,
@@ -330,9 +331,10 @@ def extras_loop(ctx, steps, device, local):
     shape = ctx["shape"]
     T, d, d_ff, E, k = shape
     x, Wg, bias, W1, W3, W2 = (inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
-    gen = torch.Generator(device=device)
-    gen.manual_seed(5)
-    gamma = (1 + 0.2 * torch.randn(d, generator=gen, device=device)).to(torch.bfloat16)
+    # gamma = 1: the normalisation then only rescales each row, which leaves every
+    # token's top-k and so the experts' loads (and the GEMMs' tiles) as in the
+    # plain layer, so the difference measures the cost of the block's edges
+    gamma = torch.ones(d, dtype=torch.bfloat16, device=device)
     eb = expert_biases(E, d, d_ff, seed=6, device=device)
     ws_b = moe.workspace(moe.moe_block_workspace_bytes(shape), device)
     H = torch.empty(T, d, dtype=torch.bfloat16, device=device)
@@ -371,7 +373,8 @@ def extras_loop(ctx, steps, device, local):
     out["bias_minus_plain_ms"] = round(out["forward_bias_ms"] - out["plain_ms"], 4)
     out["clocks"] = clocks
     out["note"] = ("same batch, calls interleaved step by step (plain, block, bias, aux); block = "
-                   "RMSNorm + layer + residual; bias = expert Linear biases b1, b3, b2; aux = "
+                   "RMSNorm (gamma = 1, so the routing and expert loads equal the plain layer's) "
+                   "+ layer + residual; bias = expert Linear biases b1, b3, b2; aux = "
                    "load-balancing term over the T x E logits")
     return out
 
@@ -470,6 +473,53 @@ def oracle_sample(inp, seconds, device_inputs=True):
                       f"experts, combine) in fp64, {dt:.1f} s wall"}, host
 
 
+def _omp_threads(n):
+    """Sets the OpenMP thread count of this process's runtime (the oracle's)."""
+    import ctypes
+    try:
+        ctypes.CDLL("libgomp.so.1").omp_set_num_threads(int(n))
+        return True
+    except OSError:
+        return False
+
+
+def oracle_per_config():
+    """The oracle's full forward (expert-major loop, fp64) on the tiny and
+    quarter-width workloads, on all host cores and on one core (quarter on one
+    core: a 64-token sample through the per-token loop); about 10 s in all."""
+    import numpy as np
+
+    import oracle
+    from sparse_mixture_experts_05_b200.inputs import workload_inputs
+    oracle.build()
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    out = {}
+    for name in ("tiny", "quarter"):
+        inp = workload_inputs(name)
+        T, d, d_ff, E, k = inp["shape"]
+        args = (inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k)
+        runs = [("all_cores", cores, None)]
+        runs.append(("one_core", 1, None if name == "tiny" else 64))
+        for label, threads, sample in runs:
+            if not _omp_threads(threads):
+                continue
+            t0 = time.perf_counter()
+            if sample is None:
+                oracle.forward(*args)
+                n = T
+            else:
+                toks = np.arange(0, T, T // sample, dtype=np.int32)[:sample]
+                oracle.forward_tokens(toks, *args)
+                n = len(toks)
+            dt = time.perf_counter() - t0
+            out[f"{name}_{label}"] = {
+                "tokens_per_s": round(n / dt, 2), "threads": threads, "seconds": round(dt, 3),
+                "what": ("full forward, expert-major loop" if sample is None else
+                         f"{n} of {T} tokens, per-token loop")}
+    _omp_threads(cores)
+    return out
+
+
 def run_ours(a):
     import torch
 
@@ -542,7 +592,10 @@ def run_ours(a):
         "ms_per_step_profiled": round(p_max_ms, 4),
         "timing": ("value and ms_per_step: moe_forward between two CUDA events per step; "
                    "kernel_ms, ms_per_step_profiled and the roofline: a second timed pass of "
-                   "the same steps through moe_forward_profiled (events between the launches)"),
+                   "the same steps through moe_forward_profiled (events between the launches); "
+                   "an event between two launches also takes away their programmatic overlap, "
+                   "so each kernel_ms entry includes that kernel's start latency (a few us, "
+                   "most visible on the small kernels)"),
         "tflops_layer": round(alg["flops_total"] / (max_ms / 1000) / 1e12, 1),
         "bracket_ms_incl_flush": round(bracket_ms, 3),
     }
@@ -558,12 +611,18 @@ def run_ours(a):
         # the skewed prefill (T = 16384, biased router): ~9 ms a step
         line["skew"] = secondary_workload("skew", min(a.steps, 10), a.warmup, device, rank,
                                           local, pg, peaks)
+        # the quarter-width and tiny workloads (~0.1 and ~0.03 ms a step)
+        for name in ("quarter", "tiny"):
+            line[name] = secondary_workload(name, max(a.steps, 40), a.warmup, device, rank,
+                                            local, pg, peaks)
 
     if world == 1 and rank == 0 and not a.no_cpu_baseline:
         from sparse_mixture_experts_05_b200.inputs import make_inputs
         w = workload(a.workload, a.tokens, a.experts)
         inp = make_inputs(w.T, w.d, w.d_ff, w.E, w.k, w.seed, bias=w.skew_bias, device=device)
         cb, _ = oracle_sample(inp, a.cpu_seconds)
+        if a.workload == "prefill" and not a.no_secondary:
+            cb["per_config"] = oracle_per_config()
         line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -59,13 +59,17 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
     if (lane <= kMaxExperts) s_pos[warp][lane] = 0;
     __syncwarp();
     // pass 1: per-warp counts (the ids of kBatch groups are loaded before any is
-    // used, so their load latencies overlap)
+    // used, so their load latencies overlap).  When the warp's run fits in one
+    // batch (T*k <= 8192) pass 2 reuses the ids kept in registers.
+    const bool one_batch = j1 - j0 <= 32 * kBatch;
+    int kept[kBatch];
     for (int base = j0; base < j1; base += 32 * kBatch) {
         int ids[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int j = base + u * 32 + lane;
             ids[u] = j < j1 ? idx[j] : -1;
+            kept[u] = ids[u];
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
@@ -119,7 +123,7 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int j = base + u * 32 + lane;
-            ids[u] = j < j1 ? idx[j] : -1;
+            ids[u] = one_batch ? kept[u] : (j < j1 ? idx[j] : -1);
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {

@@ -84,6 +84,7 @@ struct Params {
     int group_m;             // m-tiles per rasterisation group (see decode_tile_rows)
     const float* bias_a;     // GEMM1: b1 [E, n_out]; GEMM2: b2 [E, n_out]; or nullptr
     const float* bias_b;     // GEMM1: b3 [E, n_out]; or nullptr
+    int halves_inline;       // pair kernel: half tiles in place (1) or after all full tiles (0)
 };
 
 // Tiles are dealt round-robin to `active` workers (CTAs, or CTA pairs): the
@@ -571,19 +572,31 @@ constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + kEpiBy
 constexpr int kPairMinRows = 512;
 constexpr int kPairMinRounds = 8;
 
-// Tile of the pair enumeration: ids [0, F) are full tiles (expert-major, in
-// the rasterisation groups of decode_tile_rows over `s_full`), ids [F, F + H)
-// half tiles (expert-major, n fastest).
+// Tile of the pair enumeration, in one of two orders.
+//  - Half tiles last (halves_inline = 0): ids [0, F) are full tiles
+//    (expert-major, in the rasterisation groups of decode_tile_rows over
+//    s_full), ids [F, F + H) half tiles (expert-major, n fastest).  Dealt
+//    round-robin, the half tiles then go first to the pairs that got one full
+//    tile fewer: the better balance when there are few rounds of tiles.
+//  - Half tiles in place (halves_inline = 1): an expert's half m-tile is its
+//    last m-tile (decode_tile_rows over s_mt = full + half m-tiles), so the half
+//    tile of column n runs right after the full tiles of column n, while that
+//    column's weight slice is still in L2; a tile of at most 128 rows is a half
+//    tile.  The better DRAM traffic when there are many rounds of tiles.
 struct PairTile {
     TileInfo ti;
     bool half;
 };
 
 __device__ __forceinline__ PairTile decode_pair_tile(int id, int F, const int* s_full,
-                                                     const int* s_half, const int* off,
-                                                     int n_tiles, int n_tile_out, int group_m) {
+                                                     const int* s_half, const int* s_mt,
+                                                     const int* off, int n_tiles, int n_tile_out,
+                                                     int group_m, bool inline_halves) {
     PairTile pt;
-    if (id < F) {
+    if (inline_halves) {
+        pt.ti = decode_tile_rows(id, s_mt, off, n_tiles, n_tile_out, kPM, group_m);
+        pt.half = pt.ti.rows <= kPHalf;
+    } else if (id < F) {
         pt.ti = decode_tile_rows(id, s_full, off, n_tiles, n_tile_out, kPM, group_m);
         pt.half = false;
     } else {
@@ -631,6 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __shared__ int s_off[kMaxE + 1];
     __shared__ int s_full[kMaxE + 1];
     __shared__ int s_half[kMaxE + 1];
+    __shared__ int s_mt[kMaxE + 1];
     __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5;
@@ -671,6 +685,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int nf = 0, nh = 0;
         s_full[0] = 0;
         s_half[0] = 0;
+        s_mt[0] = 0;
         for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
         for (int e = 0; e < p.E; ++e) {
             const int cnt = max(0, s_off[e + 1] - s_off[e]);
@@ -679,6 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             nh += (rem > 0 && rem <= kPHalf) ? 1 : 0;
             s_full[e + 1] = nf;
             s_half[e + 1] = nh;
+            s_mt[e + 1] = nf + nh;
         }
     }
     tc_fence_before_sync();
@@ -688,8 +704,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = tmem_slot;
 
     const int n_tiles = p.n_out / p.n_tile_out;
-    const int F = s_full[p.E] * n_tiles;
-    const int H = s_half[p.E] * n_tiles;
+    const bool inl = p.halves_inline != 0;
+    // for the deal, in-place half tiles count among the F tiles (no separate H)
+    const int F = (inl ? s_mt[p.E] : s_full[p.E]) * n_tiles;
+    const int H = inl ? 0 : s_half[p.E] * n_tiles;
     const int kb_count = p.K / kBK;
     const int boxes = p.n_boxes;  // B boxes per CTA per stage
 
@@ -705,8 +723,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int i = 0; ok; ++i) {
                 const int id = deal_pair_tile(i, pair, npairs, F, H);
                 if (id < 0) break;
-                const PairTile pt = decode_pair_tile(id, F, s_full, s_half, s_off, n_tiles,
-                                                     p.n_tile_out, p.group_m);
+                const PairTile pt = decode_pair_tile(id, F, s_full, s_half, s_mt, s_off, n_tiles,
+                                                     p.n_tile_out, p.group_m, inl);
                 const CUtensorMap* am = pt.half ? &tmA64 : &tmA;
                 const int my_row0 = pt.ti.row0 + (int)rank * (pt.half ? kPHalf / 2 : kBM);
                 const uint32_t tx_pair =
@@ -769,7 +787,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int i = 0; ok; ++i) {
                 const int id = deal_pair_tile(i, pair, npairs, F, H);
                 if (id < 0) break;
-                const uint32_t idesc = id >= F ? idesc_half : idesc_full;
+                const bool half = inl ? decode_tile_rows(id, s_mt, s_off, n_tiles, p.n_tile_out,
+                                                         kPM, p.group_m).rows <= kPHalf
+                                      : id >= F;
+                const uint32_t idesc = half ? idesc_half : idesc_full;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns) || s_abort) {
                     record_error(p.err, kDeviceTimeoutBase | kRoleMma);
                     ok = false;
@@ -819,8 +840,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = 0;; ++i) {
             const int id = deal_pair_tile(i, pair, npairs, F, H);
             if (id < 0) break;
-            const PairTile pt = decode_pair_tile(id, F, s_full, s_half, s_off, n_tiles,
-                                                 p.n_tile_out, p.group_m);
+            const PairTile pt = decode_pair_tile(id, F, s_full, s_half, s_mt, s_off, n_tiles,
+                                                 p.n_tile_out, p.group_m, inl);
             const bool got = mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns);
             if (!got || s_abort) {
                 if (!got) record_error(p.err, kDeviceTimeoutBase | kRoleEpilogue);
@@ -1058,14 +1079,17 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     // upper bound on the number of tiles of either kind
     auto mtiles = [&](int tile_rows) { return (R + tile_rows - 1) / tile_rows + 2 * s.E; };
     // m-tiles per rasterisation group: as many as keep the group's activation
-    // rows (tile_rows x K bf16 each) within 16 MB.  The 126 MB L2 is split over
-    // the two dies, and the weight slices of the column tiles in flight stream
-    // through it too; on the skewed batch (experts of up to 33 pair m-tiles)
-    // 16 MB groups ran the expert GEMMs 2.5 % faster than 48 MB groups, and the
-    // prefill batch's experts (4 m-tiles) fit either way.
+    // rows (tile_rows x K bf16 each) within 32 MB of the 126 MB L2, and at
+    // least 2048 rows.  About 74 tiles run at once; a group of g m-tiles spreads
+    // them over 74 / g column tiles, whose weight slices are read from DRAM once
+    // per group, so the traffic is least near g = 8-16.  Measured DRAM bytes of
+    // the skewed batch (same box): GEMM1 (K = 4096) 6.2 GB with 16 m-tiles, 7.0
+    // with 8, 11.3 with 4; GEMM2 (K = 14336) 6.2 GB with 8, 6.9 with 4 (the
+    // 32 MB budget alone).  The step time moved by less than 1 %.
     auto group_rows = [](int tile_rows, int K) {
         const int64_t per_tile = (int64_t)tile_rows * K * 2;
-        return (int)std::max<int64_t>(1, (int64_t(16) << 20) / per_tile);
+        const int by_bytes = (int)std::max<int64_t>(1, (int64_t(32) << 20) / per_tile);
+        return std::max(by_bytes, 2048 / tile_rows);
     };
 
     Params p1{};
@@ -1086,6 +1110,10 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
     p1.bias_a = b1;
     p1.bias_b = b3;
+    // GEMM1 at the sizes that run it on pairs has dozens of tile rounds, so its
+    // half tiles go in place (next to their column's full tiles, sharing the
+    // weight slice in L2); GEMM2 has few rounds and keeps them last for balance.
+    p1.halves_inline = 0;
     // weight boxes: W1 / W3 chunks per copy = half of the CTA's B boxes
     const uint32_t ch1 = (uint32_t)p1.n_boxes / 2;
     if (!make_weight_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1) ||
@@ -1108,6 +1136,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.group_m = group_rows(pairs2 ? kPM : kBM, s.d_ff);
     p2.bias_a = b2;
     p2.bias_b = nullptr;
+    p2.halves_inline = 0;
     if (!make_weight_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, (uint32_t)p2.n_boxes))
         return MOE_ERR_CUDA;
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);

@@ -19,10 +19,11 @@
 // depends only on C and d, so results are deterministic and a caller that runs
 // one batch in token chunks can pass the whole batch's C.
 //
-// W_r staging.  W_r's rows (8 experts = 16 bytes per row and 8-expert plane)
-// are copied as they are, with 16-byte asynchronous copies, into shared memory,
-// row r of a 32-row k block at 16-byte slot r ^ (((r >> 3) & 3) << 1): the copy
-// needs no registers and overlaps the first x loads.  B fragments come out of
+// W_r staging.  Each warp copies the W_r rows of its own k range (8 experts =
+// 16 bytes per row and 8-expert plane) as they are, with 16-byte asynchronous
+// copies, into shared memory, row r of a 32-row k block at 16-byte slot
+// r ^ (((r >> 3) & 3) << 1): the copy needs no registers, overlaps the warp's
+// first x loads, and the warp waits only for its own copies.  B fragments come out of
 // it with ldmatrix .trans, whose per-lane row addresses pick the rows in the
 // order of the k permutation below; the slot swizzle makes the eight rows of
 // every 8x8 matrix fall in distinct bank groups.
@@ -190,34 +191,38 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int KS = C * kWarps;
     const int rows_cap = ((nkb + C - 1) / C) * 32;
     const int cta_kb0 = (rank * nkb) / C;
-    const int cta_rows = ((((rank + 1) * nkb) / C) - cta_kb0) * 32;
     const uint32_t s_w = sm100::smem_u32(smem);
     const uint32_t s_part = s_w + (uint32_t)(NT * rows_cap * 16);
     grid_dependency_wait();
 
-    // Stage this CTA's rows of W_r, plane by plane (8 experts per plane).
-    if ((E & 7) == 0) {
-        for (int i = tid; i < NT * cta_rows; i += kThreads) {
-            const int nt = i / cta_rows;
-            const int r = i - nt * cta_rows;
-            cp_async_16(s_w + (uint32_t)((nt * rows_cap + w_slot(r)) * 16),
-                        wg + (int64_t)(cta_kb0 * 32 + r) * E + nt * 8);
-        }
-    } else {
-        for (int i = tid; i < NT * cta_rows * 8; i += kThreads) {
-            const int j = i & 7;
-            const int rest = i >> 3;
-            const int nt = rest / cta_rows;
-            const int r = rest - nt * cta_rows;
-            const int n = nt * 8 + j;
-            const uint16_t v = n < E ? wg[(int64_t)(cta_kb0 * 32 + r) * E + n] : (uint16_t)0;
-            reinterpret_cast<uint16_t*>(smem)[(nt * rows_cap + w_slot(r)) * 8 + j] = v;
-        }
-    }
-
     const int q = rank * kWarps + warp;          // this warp's k range
     const int kb_lo = (q * nkb) / KS;
     const int kb_hi = ((q + 1) * nkb) / KS;
+    // Each warp stages the W_r rows of its own k range, plane by plane (8
+    // experts per plane), so it waits only for its own copies (no block barrier).
+    {
+        const int r0 = (kb_lo - cta_kb0) * 32;
+        const int nr = (kb_hi - kb_lo) * 32;
+        if ((E & 7) == 0) {
+            for (int i = lane; i < NT * nr; i += 32) {
+                const int nt = i / nr;
+                const int r = r0 + i - nt * nr;
+                cp_async_16(s_w + (uint32_t)((nt * rows_cap + w_slot(r)) * 16),
+                            wg + (int64_t)(cta_kb0 * 32 + r) * E + nt * 8);
+            }
+        } else {
+            for (int i = lane; i < NT * nr * 8; i += 32) {
+                const int j = i & 7;
+                const int rest = i >> 3;
+                const int nt = rest / nr;
+                const int r = r0 + rest - nt * nr;
+                const int n = nt * 8 + j;
+                const uint16_t v = n < E ? wg[(int64_t)(cta_kb0 * 32 + r) * E + n] : (uint16_t)0;
+                reinterpret_cast<uint16_t*>(smem)[(nt * rows_cap + w_slot(r)) * 8 + j] = v;
+            }
+        }
+    }
+
     // ldmatrix: lane supplies row i = lane & 7 of matrix m = lane >> 3, i.e. row
     // 8 (i >> 1) + 2 m + (i & 1) of the k block
     const int lrow = 8 * ((lane & 7) >> 1) + 2 * (lane >> 3) + (lane & 1);
@@ -246,9 +251,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                     a1[j] = v1 ? __ldg(x1 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
                 }
             }
-            if (first && it == 0) {  // W_r must have landed (every warp passes here once)
+            if (first && it == 0) {  // this warp's W_r rows must have landed
                 cp_async_wait_all();
-                __syncthreads();
+                __syncwarp();
             }
 #pragma unroll
             for (int j = 0; j < kGroup; ++j) {
@@ -273,22 +278,37 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int nt = 0; nt < NT; ++nt) mine[nt] = make_float4(c[nt][0], c[nt][1], c[nt][2], c[nt][3]);
         sm100::cluster_sync_all();
         if (rank == 0 && warp == 0) {
+            // partial sums of ranges q = 0 .. KS-1, added left to right; the loads
+            // of a batch of ranges are issued before any is added (a remote
+            // shared-memory load takes hundreds of cycles)
+            constexpr int kBatch = NT == 1 ? kWarps : (NT == 2 ? kWarps / 2 : kWarps / 4);
             float v[NT][4];
             const uint32_t buf = s_part + (uint32_t)(((it & 1) * kWarps * 32 + lane) * NT * 16);
-            for (int qq = 0; qq < KS; ++qq) {
-                const uint32_t local = buf + (uint32_t)((qq % kWarps) * 32 * NT * 16);
-                const uint32_t src = sm100::map_to_cta(local, (uint32_t)(qq / kWarps));
+            for (int cc = 0; cc < C; ++cc) {
+                const uint32_t src = sm100::map_to_cta(buf, (uint32_t)cc);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const float4 p = ld_shared_cluster_f4(src + nt * 16);
-                    if (qq == 0) {
-                        v[nt][0] = p.x; v[nt][1] = p.y; v[nt][2] = p.z; v[nt][3] = p.w;
-                    } else {
-                        v[nt][0] = __fadd_rn(v[nt][0], p.x);
-                        v[nt][1] = __fadd_rn(v[nt][1], p.y);
-                        v[nt][2] = __fadd_rn(v[nt][2], p.z);
-                        v[nt][3] = __fadd_rn(v[nt][3], p.w);
-                    }
+                for (int w0 = 0; w0 < kWarps; w0 += kBatch) {
+                    float4 p[kBatch][NT];
+#pragma unroll
+                    for (int w = 0; w < kBatch; ++w)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            p[w][nt] = ld_shared_cluster_f4(
+                                src + (uint32_t)(((w0 + w) * 32 * NT + nt) * 16));
+#pragma unroll
+                    for (int w = 0; w < kBatch; ++w)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            if (cc == 0 && w0 + w == 0) {
+                                v[nt][0] = p[w][nt].x; v[nt][1] = p[w][nt].y;
+                                v[nt][2] = p[w][nt].z; v[nt][3] = p[w][nt].w;
+                            } else {
+                                v[nt][0] = __fadd_rn(v[nt][0], p[w][nt].x);
+                                v[nt][1] = __fadd_rn(v[nt][1], p[w][nt].y);
+                                v[nt][2] = __fadd_rn(v[nt][2], p[w][nt].z);
+                                v[nt][3] = __fadd_rn(v[nt][3], p[w][nt].w);
+                            }
+                        }
                 }
             }
             if (bias) {
