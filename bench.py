@@ -331,17 +331,25 @@ def extras_loop(ctx, steps, device, local):
     shape = ctx["shape"]
     T, d, d_ff, E, k = shape
     x, Wg, bias, W1, W3, W2 = (inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
-    # gamma = 1: the normalisation then only rescales each row, which leaves every
-    # token's top-k and so the experts' loads (and the GEMMs' tiles) as in the
-    # plain layer, so the difference measures the cost of the block's edges
-    gamma = torch.ones(d, dtype=torch.bfloat16, device=device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(5)
+    gamma = (1 + 0.2 * torch.randn(d, generator=gen, device=device)).to(torch.bfloat16)
     eb = expert_biases(E, d, d_ff, seed=6, device=device)
     ws_b = moe.workspace(moe.moe_block_workspace_bytes(shape), device)
     H = torch.empty(T, d, dtype=torch.bfloat16, device=device)
     idx, _, logits = moe.moe_route(shape, x, Wg, bias, want_logits=True)
+    # the block's normalised rows u (left in its workspace for the scatter): the
+    # plain layer on u routes exactly as the block does, so block - plain-on-u
+    # is the cost of the edges alone (RMSNorm inside the router, residual in
+    # the combine) with the same expert loads and GEMM tiles
+    moe.moe_block_forward(shape, x, gamma, Wg, bias, W1, W3, W2, H=H, ws=ws_b)
+    off = moe.moe_forward_workspace_bytes(shape)
+    u = ws_b[off:off + T * d * 2].view(torch.bfloat16).view(T, d).clone()
     calls = {
         "plain_ms": lambda: moe.moe_forward(shape, x, Wg, bias, W1, W3, W2, y=ctx["y"],
                                             ws=ctx["ws"]),
+        "plain_on_u_ms": lambda: moe.moe_forward(shape, u, Wg, bias, W1, W3, W2, y=ctx["y"],
+                                                 ws=ctx["ws"]),
         "block_forward_ms": lambda: moe.moe_block_forward(shape, x, gamma, Wg, bias, W1, W3, W2,
                                                           H=H, ws=ws_b),
         "forward_bias_ms": lambda: moe.moe_forward_bias(shape, x, Wg, bias, W1, W3, W2, eb,
@@ -369,13 +377,14 @@ def extras_loop(ctx, steps, device, local):
     if moe.moe_read_device_status(ws_b) != moe.MOE_OK:
         raise RuntimeError("device status error in the block forward")
     out = {name: round(statistics.mean(v), 4) for name, v in times.items()}
-    out["block_minus_plain_ms"] = round(out["block_forward_ms"] - out["plain_ms"], 4)
+    out["block_minus_plain_on_u_ms"] = round(out["block_forward_ms"] - out["plain_on_u_ms"], 4)
     out["bias_minus_plain_ms"] = round(out["forward_bias_ms"] - out["plain_ms"], 4)
     out["clocks"] = clocks
-    out["note"] = ("same batch, calls interleaved step by step (plain, block, bias, aux); block = "
-                   "RMSNorm (gamma = 1, so the routing and expert loads equal the plain layer's) "
-                   "+ layer + residual; bias = expert Linear biases b1, b3, b2; aux = "
-                   "load-balancing term over the T x E logits")
+    out["note"] = ("same batch, calls interleaved step by step (plain, plain on u, block, bias, "
+                   "aux); block = RMSNorm inside the router + layer + residual in the combine, "
+                   "gamma ~ 1 + N(0, 0.04); plain on u = the layer on the block's own "
+                   "normalised rows (same routing and GEMM tiles as the block); bias = expert "
+                   "Linear biases b1, b3, b2; aux = load-balancing term over the T x E logits")
     return out
 
 

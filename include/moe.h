@@ -214,8 +214,11 @@ int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float
  *   gamma [d] bf16: RMSNorm_2 scale; eps >= 0 (rms_norm_eps, 1e-5 for Mixtral) (in)
  *   Wg, bias, W1, W3, W2 as for moe_forward (in);  H [T,d] bf16 (out)
  *   ws: >= moe_block_workspace_bytes(s) bytes of device memory
- * The normalised rows are rounded to bf16 (the layer's input); the residual is
- * added in float32 to the combined expert outputs before the one rounding of H.
+ * The normalised rows are rounded to bf16 (the layer's input); the router
+ * computes them while it reads U and leaves them in the workspace, at byte
+ * offset moe_forward_workspace_bytes(s) ([T,d] bf16), for the dispatch.  The
+ * residual is added in float32 to the combined expert outputs before the one
+ * rounding of H.
  */
 size_t moe_block_workspace_bytes(moe_shape s);
 int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, const void* Wg,

@@ -12,7 +12,6 @@
 #include <mutex>
 
 #include "aux_loss.cuh"
-#include "block.cuh"
 #include "combine.cuh"
 #include "common.cuh"
 #include "dispatch.cuh"
@@ -102,6 +101,7 @@ struct FwdOptions {
     bool clear_status = true;        // the index kernel zeroes the status word first
     int stall_after = -1;            // test hook: expert producer stops after this many stages
     uint64_t timeout_ns = kDefaultWaitTimeoutNs;  // bound on every device wait
+    const RouterNorm* norm = nullptr;  // block edge: x is U, the router forms u = RMSNorm_2(U)
 };
 
 // Records events[i] (when given) between the launches: 0 before the router, 1
@@ -125,13 +125,14 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     float* o = at<float>(ws, L.o);
     int* status = at<int>(ws, L.hdr);
     if (!mark(0)) return MOE_ERR_CUDA;
-    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_cluster);
+    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_cluster, opt.norm);
     if (rc) return rc;
     if (!mark(1)) return MOE_ERR_CUDA;
     rc = launch_dispatch_index(s, idx, offsets, perm, inv, opt.clear_status ? status : nullptr, st);
     if (rc) return rc;
     if (!mark(2)) return MOE_ERR_CUDA;
-    rc = launch_dispatch_scatter(s, x, inv, xs, st);
+    // the experts' rows: the layer input, or the router's normalised rows u
+    rc = launch_dispatch_scatter(s, opt.norm ? opt.norm->u : x, inv, xs, st);
     if (rc) return rc;
     if (!mark(3)) return MOE_ERR_CUDA;
     rc = expert_gemms(s, xs, offsets, W1, W3, W2, h, o, status, opt.timeout_ns, opt.stall_after,
@@ -474,12 +475,17 @@ int moe_block_forward(moe_shape s, const void* U, const void* gamma, float eps, 
         return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_block_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    void* u = static_cast<char*>(ws) + moe_forward_workspace_bytes(s);
-    rc = launch_rmsnorm(s, U, gamma, eps, u, st);
-    if (rc) return rc;
+    // RMSNorm_2 runs inside the router (which reads every row of U anyway) and
+    // leaves u in the workspace for the scatter; the residual is added in the
+    // combine.
+    RouterNorm norm;
+    norm.gamma = gamma;
+    norm.eps = eps;
+    norm.u = static_cast<char*>(ws) + moe_forward_workspace_bytes(s);
     FwdOptions opt;
     opt.residual = U;
-    return forward_impl(s, u, Wg, bias, W1, W3, W2, H, nullptr, nullptr, ws, st, nullptr, opt);
+    opt.norm = &norm;
+    return forward_impl(s, U, Wg, bias, W1, W3, W2, H, nullptr, nullptr, ws, st, nullptr, opt);
 }
 
 int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const float* bias,

@@ -1113,7 +1113,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     // GEMM1 at the sizes that run it on pairs has dozens of tile rounds, so its
     // half tiles go in place (next to their column's full tiles, sharing the
     // weight slice in L2); GEMM2 has few rounds and keeps them last for balance.
-    p1.halves_inline = 0;
+    p1.halves_inline = 1;
     // weight boxes: W1 / W3 chunks per copy = half of the CTA's B boxes
     const uint32_t ch1 = (uint32_t)p1.n_boxes / 2;
     if (!make_weight_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1) ||

@@ -89,6 +89,36 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// RMSNorm helpers (block edge, see router_kernel's kNorm): the sum of squares of
+// 8 bf16 values added in order to ss, and bf16((x * inv) * gamma) of 8 values.
+__device__ __forceinline__ float sum_squares8(const uint4& v, float ss) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float lo = bf16_lo(w[j]), hi = bf16_hi(w[j]);
+        ss = __fadd_rn(ss, __fmul_rn(lo, lo));
+        ss = __fadd_rn(ss, __fmul_rn(hi, hi));
+    }
+    return ss;
+}
+
+__device__ __forceinline__ uint4 rms_scale8(const uint4& v, const uint4& gm, float inv) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t gw[4] = {gm.x, gm.y, gm.z, gm.w};
+    uint32_t r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        r[j] = pack_bf16x2(__fmul_rn(__fmul_rn(bf16_lo(w[j]), inv), bf16_lo(gw[j])),
+                           __fmul_rn(__fmul_rn(bf16_hi(w[j]), inv), bf16_hi(gw[j])));
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
 // 16-byte slot of row r (local to the CTA's staged range) of a W_r plane.
 __device__ __forceinline__ int w_slot(int r) { return r ^ (((r >> 3) & 3) << 1); }
 
@@ -174,13 +204,28 @@ __device__ __noinline__ void select_and_store(float (&v)[NT][4], int tile, int T
 
 // Dynamic shared memory: NT planes of W_r rows [rows_cap][16 bytes], then the
 // partial sums [2 buffers][kWarps][32 lanes][NT] float4.
-template <int NT>
+//
+// kNorm (the block edge RMSNorm_2 of the Mixtral page's block equation, fused
+// here because the router reads every row of its input anyway): x is the
+// residual stream U, and the layer's input is u = bf16((U * inv) * gamma) with
+// inv = 1 / sqrt(mean_j U_j^2 + eps) per row.  Per token tile, pass A reads the
+// warp's k range and adds the squares per row (in order within a lane, then
+// over the quad, then over the 8 C ranges in range order after a cluster
+// barrier, every warp for its own rows); pass B reads the range again (from
+// L2), forms u, writes it to u_out (the scatter's input) and feeds the same u to
+// the MMAs.
+template <int NT, bool kNorm>
 __global__ void __launch_bounds__(kThreads, 2)
     router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
                   const float* __restrict__ bias, int T, int d, int E, int k, int C,
                   int32_t* __restrict__ idx, float* __restrict__ gate,
-                  float* __restrict__ logits) {
+                  float* __restrict__ logits, const uint16_t* __restrict__ gamma, float eps,
+                  uint16_t* __restrict__ u_out) {
     extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ float s_ss[kWarps][16];  // kNorm: per-warp sums of squares of the tile's rows
+    // k blocks whose x loads are issued together (halved when normalising, which
+    // holds more per lane: the scaled u and the gamma chunks)
+    constexpr int kG = kNorm ? kGroup / 2 : kGroup;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -241,14 +286,87 @@ __global__ void __launch_bounds__(kThreads, 2)
         const bool v0 = r0 < T, v1 = r1 < T;
         const uint4* x0 = reinterpret_cast<const uint4*>(x + (int64_t)(v0 ? r0 : 0) * d) + t4;
         const uint4* x1 = reinterpret_cast<const uint4*>(x + (int64_t)(v1 ? r1 : 0) * d) + t4;
-        for (int kb = kb_lo, first = 1; first || kb < kb_hi; kb += kGroup, first = 0) {
-            const int n = min(kGroup, kb_hi - kb);
-            uint4 a0[kGroup], a1[kGroup];
+        float inv0 = 1.0f, inv1 = 1.0f;
+        if constexpr (kNorm) {
+            // pass A: sums of squares of rows r0 and r1 over this warp's range
+            float ss0 = 0.0f, ss1 = 0.0f;
+            for (int kb = kb_lo; kb < kb_hi; kb += kG) {
+                const int n = min(kG, kb_hi - kb);
+                uint4 a0[kG], a1[kG];
 #pragma unroll
-            for (int j = 0; j < kGroup; ++j) {
+                for (int j = 0; j < kG; ++j) {
+                    if (j < n) {
+                        a0[j] = v0 ? __ldg(x0 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
+                        a1[j] = v1 ? __ldg(x1 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kG; ++j) {
+                    if (j < n) {
+                        ss0 = sum_squares8(a0[j], ss0);
+                        ss1 = sum_squares8(a1[j], ss1);
+                    }
+                }
+            }
+            // the four lanes of a quad hold the same rows: fl(a+b) = fl(b+a), so
+            // every lane of the quad gets the same bits
+            ss0 = __fadd_rn(ss0, __shfl_xor_sync(0xffffffffu, ss0, 1));
+            ss0 = __fadd_rn(ss0, __shfl_xor_sync(0xffffffffu, ss0, 2));
+            ss1 = __fadd_rn(ss1, __shfl_xor_sync(0xffffffffu, ss1, 1));
+            ss1 = __fadd_rn(ss1, __shfl_xor_sync(0xffffffffu, ss1, 2));
+            if (t4 == 0) {
+                s_ss[warp][g] = ss0;
+                s_ss[warp][g + 8] = ss1;
+            }
+            sm100::cluster_sync_all();
+            // the row totals over all 8 C ranges, in range order (loads of a CTA
+            // issued together)
+            float tot0 = 0.0f, tot1 = 0.0f;
+            const uint32_t ss_base = sm100::smem_u32(&s_ss[0][0]);
+            for (int cc = 0; cc < C; ++cc) {
+                const uint32_t src = sm100::map_to_cta(ss_base, (uint32_t)cc);
+#pragma unroll
+                for (int w0 = 0; w0 < kWarps; w0 += 4) {
+                    float p0[4], p1[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        p0[w] = ld_shared_cluster_f32(src + (uint32_t)(((w0 + w) * 16 + g) * 4));
+                        p1[w] = ld_shared_cluster_f32(src + (uint32_t)(((w0 + w) * 16 + g + 8) * 4));
+                    }
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        tot0 = (cc == 0 && w0 + w == 0) ? p0[w] : __fadd_rn(tot0, p0[w]);
+                        tot1 = (cc == 0 && w0 + w == 0) ? p1[w] : __fadd_rn(tot1, p1[w]);
+                    }
+                }
+            }
+            inv0 = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot0, (float)d), eps)));
+            inv1 = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot1, (float)d), eps)));
+        }
+        for (int kb = kb_lo, first = 1; first || kb < kb_hi; kb += kG, first = 0) {
+            const int n = min(kG, kb_hi - kb);
+            uint4 a0[kG], a1[kG];
+#pragma unroll
+            for (int j = 0; j < kG; ++j) {
                 if (j < n) {
                     a0[j] = v0 ? __ldg(x0 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
                     a1[j] = v1 ? __ldg(x1 + (kb + j) * 4) : make_uint4(0, 0, 0, 0);
+                }
+            }
+            if constexpr (kNorm) {
+                // pass B: u = bf16((x * inv) * gamma), stored for the scatter
+                const uint4* g4 = reinterpret_cast<const uint4*>(gamma) + t4;
+                uint4* u0 = reinterpret_cast<uint4*>(u_out + (int64_t)(v0 ? r0 : 0) * d) + t4;
+                uint4* u1 = reinterpret_cast<uint4*>(u_out + (int64_t)(v1 ? r1 : 0) * d) + t4;
+#pragma unroll
+                for (int j = 0; j < kG; ++j) {
+                    if (j < n) {
+                        const uint4 gm = __ldg(g4 + (kb + j) * 4);
+                        a0[j] = rms_scale8(a0[j], gm, inv0);
+                        a1[j] = rms_scale8(a1[j], gm, inv1);
+                        if (v0) u0[(kb + j) * 4] = a0[j];
+                        if (v1) u1[(kb + j) * 4] = a1[j];
+                    }
                 }
             }
             if (first && it == 0) {  // this warp's W_r rows must have landed
@@ -256,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 __syncwarp();
             }
 #pragma unroll
-            for (int j = 0; j < kGroup; ++j) {
+            for (int j = 0; j < kG; ++j) {
                 if (j < n) {
                     const uint32_t blk = s_w + (uint32_t)((kb + j - cta_kb0) * 32 * 16) + lane_off;
 #pragma unroll
@@ -343,7 +461,8 @@ int router_cluster(const moe_shape& s) {
 }
 
 int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
-                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int cluster) {
+                  int32_t* idx, float* gate, float* logits, cudaStream_t stream, int cluster,
+                  const RouterNorm* norm) {
     using namespace router;
     if (s.T == 0) return MOE_OK;
     const int NT = (s.E + 7) / 8;
@@ -360,6 +479,9 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
     const int nclusters = std::max(1, std::min(ntiles, (2 * sms) / C));
     const uint16_t* xp = static_cast<const uint16_t*>(x);
     const uint16_t* wp = static_cast<const uint16_t*>(Wg);
+    const uint16_t* gp = norm ? static_cast<const uint16_t*>(norm->gamma) : nullptr;
+    const float eps = norm ? norm->eps : 0.0f;
+    uint16_t* up = norm ? static_cast<uint16_t*>(norm->u) : nullptr;
     auto run = [&](auto kern) {
         if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem))
             return MOE_ERR_CUDA;
@@ -378,17 +500,21 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, kern, xp, wp, bias, s.T, s.d, s.E, s.k, C, idx, gate,
-                                  logits) == cudaSuccess
+                                  logits, gp, eps, up) == cudaSuccess
                    ? MOE_OK
                    : MOE_ERR_CUDA;
     };
+#define MOE_ROUTER_CASE(N)                                                              \
+    case N:                                                                             \
+        return norm ? run(router_kernel<N, true>) : run(router_kernel<N, false>);
     switch (NT) {
-        case 1: return run(router_kernel<1>);
-        case 2: return run(router_kernel<2>);
-        case 3: return run(router_kernel<3>);
-        case 4: return run(router_kernel<4>);
+        MOE_ROUTER_CASE(1)
+        MOE_ROUTER_CASE(2)
+        MOE_ROUTER_CASE(3)
+        MOE_ROUTER_CASE(4)
         default: return MOE_ERR_UNSUPPORTED;
     }
+#undef MOE_ROUTER_CASE
 }
 
 }  // namespace moe

@@ -22,10 +22,23 @@ def _gamma(d, seed):
     return torch.from_numpy((1 + 0.2 * rng.standard_normal(d)).astype(np.float32)).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "quarter"])
+BLOCK_CASES = {
+    # the router normalises the rows itself; its cluster size (CTAs sharing a
+    # token tile's contraction) depends on T and d: 1 for tiny and ragged, 4 for
+    # the quarter-width batch, 8 for the decode-sized batch at d = 4096
+    "ragged": (77, 256, 384, 8, 2, 5, True),
+    "decode-d4096": (16, 4096, 256, 8, 2, 6, False),
+    "mid-d2048": (300, 2048, 256, 8, 2, 7, True),
+}
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "quarter", "decode-d4096", "mid-d2048"])
 def test_block_forward_matches_oracle(name):
-    inp = workload_inputs("quarter") if name == "quarter" else (
-        workload_inputs("tiny") if name == "tiny" else make_inputs(77, 256, 384, 8, 2, 5, bias=True))
+    if name in BLOCK_CASES:
+        T, d, d_ff, E, k, seed, bias = BLOCK_CASES[name]
+        inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    else:
+        inp = workload_inputs(name)
     T, d, d_ff, E, k = inp["shape"]
     gamma = _gamma(d, 7)
     dev = to_dev(inp)
@@ -52,3 +65,30 @@ def test_block_zero_down_projection_returns_the_residual_exactly():
     H = moe.moe_block_forward(inp["shape"], dev["x"], _gamma(128, 8).cuda(), dev["Wg"], None,
                               dev["W1"], dev["W3"], zero)
     assert torch.equal(H, dev["x"])
+
+
+@pytest.mark.parametrize("name", ["quarter", "decode-d4096"])
+def test_router_normalised_rows_match_oracle_rmsnorm(name):
+    """The router writes u = bf16((U * inv) * gamma) into the block workspace (right
+    after moe_forward's part) for the scatter; u equals the oracle's RMSNorm to
+    within one bf16 ulp (the float32 sum of squares is added in another order
+    than the oracle's double sum), and nearly always exactly."""
+    if name in BLOCK_CASES:
+        T, d, d_ff, E, k, seed, bias = BLOCK_CASES[name]
+        inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    else:
+        inp = workload_inputs(name)
+    T, d, d_ff, E, k = inp["shape"]
+    gamma = _gamma(d, 9)
+    dev = to_dev(inp)
+    ws = moe.workspace(moe.moe_block_workspace_bytes(inp["shape"]), "cuda")
+    moe.moe_block_forward(inp["shape"], dev["x"], gamma.cuda(), dev["Wg"], dev["bias"], dev["W1"],
+                          dev["W3"], dev["W2"], eps=1e-5, ws=ws)
+    torch.cuda.synchronize()
+    off = moe.moe_forward_workspace_bytes(inp["shape"])
+    u = ws[off:off + T * d * 2].view(torch.bfloat16).view(T, d)
+    u_ref = oracle.bf16_to_f64(oracle.rmsnorm(inp["x"], gamma, 1e-5))
+    uv = bf16_values(u)
+    diff = np.abs(uv - u_ref)
+    assert np.all(diff <= bf16_ulp(u_ref) * 1.0001 + 1e-30)
+    assert np.mean(diff > 0) < 1e-3
