@@ -571,6 +571,7 @@ constexpr int kPairStageBytes = kABytes + kPairBBoxes * kBBoxBytes;   // 32 KB
 constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + kEpiBytes + 1024;
 constexpr int kPairMinRows = 512;
 constexpr int kPairMinRounds = 8;
+constexpr int kInlineHalfRounds = 16;
 
 // Tile of the pair enumeration, in one of two orders.
 //  - Half tiles last (halves_inline = 0): ids [0, F) are full tiles
@@ -1110,10 +1111,16 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p1.group_m = group_rows(pairs1 ? kPM : kBM, s.d);
     p1.bias_a = b1;
     p1.bias_b = b3;
-    // GEMM1 at the sizes that run it on pairs has dozens of tile rounds, so its
-    // half tiles go in place (next to their column's full tiles, sharing the
-    // weight slice in L2); GEMM2 has few rounds and keeps them last for balance.
-    p1.halves_inline = 1;
+    // Half tiles go in place (next to their column's full tiles, sharing the
+    // weight slice in L2) when the launch has many rounds of pair tiles, and
+    // last (for balance) when it has few: GEMM1 at the prefill batch runs ~48
+    // rounds, GEMM2 ~7, GEMM2 at the skewed batch ~28.
+    auto inline_halves = [&](int n_cols_per_tile, int n_out) {
+        const int64_t rounds = ((int64_t)R / kPM) * (n_out / n_cols_per_tile) /
+                               std::max(1, max_pairs<true>());
+        return rounds >= kInlineHalfRounds ? 1 : 0;
+    };
+    p1.halves_inline = inline_halves(128, s.d_ff);
     // weight boxes: W1 / W3 chunks per copy = half of the CTA's B boxes
     const uint32_t ch1 = (uint32_t)p1.n_boxes / 2;
     if (!make_weight_map(&m1, W1, (uint64_t)s.E * s.d, (uint64_t)s.d_ff, ch1) ||
@@ -1136,7 +1143,7 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.group_m = group_rows(pairs2 ? kPM : kBM, s.d_ff);
     p2.bias_a = b2;
     p2.bias_b = nullptr;
-    p2.halves_inline = 0;
+    p2.halves_inline = inline_halves(p2.n_tile_out, s.d);
     if (!make_weight_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, (uint32_t)p2.n_boxes))
         return MOE_ERR_CUDA;
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);
