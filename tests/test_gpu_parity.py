@@ -31,6 +31,11 @@ CASES = {
     "single": (1, 128, 256, 8, 2, 11, False),
     "batch16": (16, 256, 384, 8, 2, 16, True),    # decode-sized: R = 32 rows over 8 experts
     "batch30": (30, 128, 512, 8, 2, 17, False),
+    # GEMM1 on CTA pairs with its half tiles in place (R = 9600 rows: about 16
+    # rounds of pair tiles), GEMM2 on pairs with its half tiles last
+    "pairs-inline": (4800, 256, 4096, 8, 2, 19, True),
+    # one expert: four full pair tiles and a 76-row half tile
+    "E1-pairs": (1100, 256, 512, 1, 1, 21, False),
 }
 
 
