@@ -7,9 +7,11 @@
 // an exclusive scan of the per-expert counts produces.
 //
 // Two launches:
-//  1. index kernel (one CTA of 1024 threads): each warp owns a contiguous run
-//     of slots; warp-wide grouping by expert id (__match_any_sync) gives counts
-//     and in-order ranks, one warp scans the per-warp counts into offsets and
+//  1. index kernel (a cluster of 1 to 8 CTAs of 1024 threads, sized so each
+//     warp owns a run of about 64 slots): each warp owns a contiguous run of
+//     slots; warp-wide grouping by expert id (__match_any_sync) gives counts and
+//     in-order ranks, the CTAs scan the per-warp counts (sharing their
+//     per-expert totals through distributed shared memory) into offsets and
 //     starting positions, and a second pass hands out positions in token order.
 //     Integer-only and deterministic (no atomics on positions).
 //  2. scatter kernel: reads each x row once and writes it to its k sorted rows
@@ -20,6 +22,7 @@
 
 #include "common.cuh"
 #include "dispatch.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace dispatch {
@@ -28,37 +31,58 @@ constexpr int kIndexThreads = 1024;  // 32 warps
 constexpr int kIndexWarps = kIndexThreads / 32;
 constexpr int kMaxExperts = 32;
 constexpr int kBatch = 8;  // groups of 32 slots whose ids are loaded together
+constexpr int kMaxIndexCluster = 8;
+constexpr int kSlotsPerWarp = 64;  // target run length per warp when choosing the cluster size
 
-// One CTA.  The T*k slots (slot j = t*k + s, ascending in t) are cut into 32
-// contiguous runs, one per warp, taken 32 slots at a time.  In each group of
-// 32 slots, __match_any_sync on the expert id gives every lane the lanes that
-// chose the same expert: their number and this lane's rank among them (lane
-// order = slot order).  Pass 1 sums the per-warp, per-expert counts; one warp
-// turns them into offsets and per-warp starting positions (expert-major, then
-// warp order); pass 2 repeats the grouping and hands out positions.  Stable
-// (slot order within each expert), deterministic, no atomics.
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ int ld_shared_cluster_s32(uint32_t addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// A cluster of C CTAs (C = 1 .. 8, chosen from T*k).  The T*k slots (slot
+// j = t*k + s, ascending in t) are cut into 32 C contiguous runs, one per warp
+// in cluster order (CTA rank, then warp), taken 32 slots at a time.  In each
+// group of 32 slots, __match_any_sync on the expert id gives every lane the
+// lanes that chose the same expert: their number and this lane's rank among
+// them (lane order = slot order).  Pass 1 sums the per-warp, per-expert counts;
+// warp e of every CTA scans expert e's counts over its 32 warps, the CTAs read
+// each other's per-expert totals through distributed shared memory (so each
+// knows the rows of every expert in earlier CTAs and in all), and the
+// per-warp starting positions follow (expert-major, then slot order); pass 2
+// repeats the grouping and hands out positions.  Stable (slot order within each
+// expert), deterministic, no atomics.
 __global__ void __launch_bounds__(kIndexThreads, 1)
     index_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                  int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
                  int32_t* __restrict__ inv, int* status_to_clear) {
     __shared__ int s_pos[kIndexWarps][kMaxExperts + 1];  // counts, then next positions
-    __shared__ int s_total[kMaxExperts];                  // rows per expert
-    __shared__ int s_base[kMaxExperts];                   // first sorted row of each expert
+    __shared__ int s_total[kMaxExperts];                  // this CTA's rows per expert
+    __shared__ int s_base[kMaxExperts];                   // first row of each expert in this CTA
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
+    const int rank = (int)sm100::cluster_ctarank();
+    const int C = (int)cluster_size();
     grid_dependency_wait();
-    if (status_to_clear && tid == 0) *status_to_clear = 0;
+    if (status_to_clear && tid == 0 && rank == 0) *status_to_clear = 0;
 
     const int n = T * k;
-    const int per_warp = ((n + kIndexWarps - 1) / kIndexWarps + 31) / 32 * 32;
-    const int j0 = min(n, warp * per_warp);
+    const int nwarps = kIndexWarps * C;
+    const int gwarp = rank * kIndexWarps + warp;
+    const int per_warp = ((n + nwarps - 1) / nwarps + 31) / 32 * 32;
+    const int j0 = min(n, gwarp * per_warp);
     const int j1 = min(n, j0 + per_warp);
     const unsigned lt_mask = (1u << lane) - 1u;
 
     if (lane <= kMaxExperts) s_pos[warp][lane] = 0;
-    __syncwarp();
-    // pass 1: per-warp counts (the ids of kBatch groups are loaded before any is
+    __syncwarp();    // pass 1: per-warp counts (the ids of kBatch groups are loaded before any is
     // used, so their load latencies overlap).  When the warp's run fits in one
     // batch (T*k <= 8192) pass 2 reuses the ids kept in registers.
     const bool one_batch = j1 - j0 <= 32 * kBatch;
@@ -73,6 +97,7 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            if (base + u * 32 >= j1) break;  // warp-uniform: past the warp's run
             const int e = ids[u];
             const bool valid = e >= 0 && e < E;
             const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);
@@ -83,7 +108,8 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
     __syncthreads();
 
     // offsets and per-warp starting positions: warp e scans expert e's counts
-    // over the 32 warps (lane = warp), then warp 0 scans the experts' totals
+    // over this CTA's 32 warps (lane = warp); then every CTA reads all CTAs'
+    // totals: rows of expert e in earlier CTAs, and in all
     {
         int excl_w = 0;
         if (warp < E) {
@@ -94,29 +120,37 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
                 const int o = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off) incl += o;
             }
-            excl_w = incl - c;  // rows of expert `warp` in warps before `lane`
+            excl_w = incl - c;  // rows of expert `warp` in this CTA's warps before `lane`
             if (lane == 31) s_total[warp] = incl;
         }
-        __syncthreads();
+        sm100::cluster_sync_all();
         if (warp == 0) {
-            const int total = lane < E ? s_total[lane] : 0;
+            int before = 0, total = 0;  // rows of expert `lane` in earlier CTAs / in all
+            if (lane < E) {
+                const uint32_t src0 = sm100::smem_u32(&s_total[lane]);
+                for (int c = 0; c < C; ++c) {
+                    const int t = ld_shared_cluster_s32(sm100::map_to_cta(src0, (uint32_t)c));
+                    if (c < rank) before += t;
+                    total += t;
+                }
+            }
             int incl = total;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int o = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off) incl += o;
             }
+            const int expert_start = incl - total;
             if (lane < E) {
-                s_base[lane] = incl - total;
-                offsets[lane] = incl - total;
+                s_base[lane] = expert_start + before;
+                if (rank == 0) offsets[lane] = expert_start;
             }
-            if (lane == 31) offsets[E] = incl;
+            if (lane == 31 && rank == 0) offsets[E] = incl;
         }
         __syncthreads();
         if (warp < E) s_pos[lane][warp] = s_base[warp] + excl_w;
     }
     __syncthreads();
-
     // pass 2: positions in slot order
     for (int base = j0; base < j1; base += 32 * kBatch) {
         int ids[kBatch];
@@ -127,6 +161,7 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            if (base + u * 32 >= j1) break;  // warp-uniform: past the warp's run
             const int j = base + u * 32 + lane;
             const bool in = j < j1;
             const int e = ids[u];
@@ -144,6 +179,8 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
             __syncwarp();
         }
     }
+    // no CTA leaves while another may still read its per-expert totals
+    sm100::cluster_sync_all();
 }
 
 // x_sorted[inv[t, s]] = x[t] for every slot s of token t; one thread per
@@ -175,8 +212,26 @@ int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offse
                           cudaStream_t stream) {
     using namespace dispatch;
     if (s.E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
-    return launch_pdl(index_kernel, dim3(1), dim3(kIndexThreads), 0, stream, idx, s.T, s.E, s.k,
-                      offsets, perm_tok, inv, status_to_clear) == cudaSuccess
+    // cluster size: enough CTAs for runs of about kSlotsPerWarp slots per warp
+    const int64_t n = (int64_t)s.T * s.k;
+    int C = 1;
+    while (C < kMaxIndexCluster && n > (int64_t)C * kIndexWarps * kSlotsPerWarp) C *= 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C);
+    cfg.blockDim = dim3(kIndexThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, index_kernel, idx, s.T, s.E, s.k, offsets, perm_tok, inv,
+                              status_to_clear) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }
