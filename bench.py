@@ -403,6 +403,9 @@ def secondary_workload(name, steps, warmup, device, rank, local, pg, peaks):
     world = 1 if pg is None else pg.get_world_size()
     out = {"workload": WORKLOAD_NAMES[name], "tokens_per_s": round(T * world / (mean / 1e3), 1),
            "ms_per_step": round(mean, 4), "steps": w_steps,
+           # for sub-millisecond steps a few host-side hiccups move the mean
+           "ms_per_step_median": round(statistics.median(ms), 4),
+           "ms_per_step_max": round(max(ms), 4),
            "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
            "ms_per_step_profiled": round(pmean, 4), "expert_rows": ctx["counts"],
            "clocks": clocks}
