@@ -246,6 +246,33 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
                        size_t ws_bytes, void* stream);
 
 /*
+ * moe_forward_hostio_batches -- moe_forward over n_batches independent batches
+ * of T tokens each with the same weights, batch b read from the host buffer
+ * x_host[b] and written to the host buffer y_host[b] (pinned memory gives
+ * asynchronous copies); the loop of a server that feeds the layer a queue of
+ * batches.  Each batch runs the whole layer once on `stream` (the weights are
+ * streamed once per batch, not once per token chunk); batch b+1's upload and
+ * batch b-1's download run on the library's two copy streams while batch b
+ * computes, through two staging slots in ws, so only the first upload and the
+ * last download are not overlapped.  y_host[b] equals moe_forward on x_host[b]
+ * bit for bit.  Everything is ordered after earlier work on `stream`, and
+ * `stream` after the last download.  The status word is cleared once, before
+ * the first batch, so an expired wait in any batch stays reported.
+ *   x_host, y_host: arrays of n_batches host pointers (none null), each buffer
+ *       T*d bf16, row-major; a buffer may appear more than once (the caller
+ *       owns the data order: y_host[b] is written when batch b's download runs).
+ *   ws: >= moe_forward_workspace_bytes(s) + 2 x-staging + 2 y-staging slots of
+ *       T*d*2 bytes; moe_forward_hostio_batches_workspace_bytes gives the figure.
+ * Errors: MOE_ERR_INVALID_ARG for n_batches < 1 or a null array or entry,
+ * MOE_ERR_WORKSPACE for a short ws; T == 0 enqueues nothing.
+ */
+size_t moe_forward_hostio_batches_workspace_bytes(moe_shape s);
+int moe_forward_hostio_batches(moe_shape s, int n_batches, const void* const* x_host,
+                               const void* Wg, const float* bias, const void* W1,
+                               const void* W3, const void* W2, void* const* y_host, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/*
  * moe_forward_hostio_stall_test -- test hook for the error path of the chunked
  * host-I/O pipeline (no counterpart on the pages).  Runs moe_forward_hostio with
  * the expert kernels' TMA producer of token chunk `stall_chunk` (0 = first;

@@ -98,7 +98,7 @@ struct FwdOptions {
     const void* residual = nullptr;  // [T, d] bf16 added before the rounding of y (block edge)
     ExpertBias eb;                   // expert Linear biases
     int router_cluster = 0;          // router cluster size, fixing its k split (0: chosen for this T)
-    bool clear_status = true;        // the index kernel zeroes the status word first
+    bool clear_status = true;        // the router (first kernel) zeroes the status word first
     int stall_after = -1;            // test hook: expert producer stops after this many stages
     uint64_t timeout_ns = kDefaultWaitTimeoutNs;  // bound on every device wait
     const RouterNorm* norm = nullptr;  // block edge: x is U, the router forms u = RMSNorm_2(U)
@@ -125,10 +125,11 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     float* o = at<float>(ws, L.o);
     int* status = at<int>(ws, L.hdr);
     if (!mark(0)) return MOE_ERR_CUDA;
-    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_cluster, opt.norm);
+    int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_cluster, opt.norm,
+                           status, opt.clear_status);
     if (rc) return rc;
     if (!mark(1)) return MOE_ERR_CUDA;
-    rc = launch_dispatch_index(s, idx, offsets, perm, inv, opt.clear_status ? status : nullptr, st);
+    rc = launch_dispatch_index(s, idx, offsets, perm, inv, st);
     if (rc) return rc;
     if (!mark(2)) return MOE_ERR_CUDA;
     // the experts' rows: the layer input, or the router's normalised rows u
@@ -194,6 +195,9 @@ int hostio_chunks(int T, int (&sizes)[kMaxHostioChunks]) {
 struct CopyStreams {
     cudaStream_t up = nullptr, down = nullptr;
     cudaEvent_t ev[2 + 2 * kMaxHostioChunks] = {};
+    // moe_forward_hostio_batches: start, x landed in slot 0/1, slot 0/1's layer
+    // done, slot 0/1's y left, end
+    cudaEvent_t evb[8] = {};
     std::mutex mu;
 };
 
@@ -209,6 +213,8 @@ CopyStreams* copy_streams() {
                   cudaStreamCreateWithFlags(&cs->down, cudaStreamNonBlocking) == cudaSuccess;
         for (auto& e : cs->ev)
             ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        for (auto& e : cs->evb)
+            ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
         if (!ok) return nullptr;  // (leaks the partial set; only on a failing device)
         per_device[dev] = cs;
     }
@@ -217,7 +223,7 @@ CopyStreams* copy_streams() {
 
 // moe_forward_hostio with an optional stall of the expert producer in chunk
 // `stall_chunk` (test hook; -1: none).  The status word is cleared once, by the
-// first chunk's index kernel: a later chunk must not erase an expired wait that
+// first chunk's router kernel: a later chunk must not erase an expired wait that
 // an earlier chunk recorded.
 int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const float* bias,
                 const void* W1, const void* W3, const void* W2, void* y_host, void* ws,
@@ -296,6 +302,61 @@ int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const fl
     return ok ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// moe_forward_hostio_batches: n independent batches through two staging slots.
+// Batch b uses slot b & 1; its upload waits until batch b-2's layer has read
+// the slot's x (so it runs while batch b-1 computes), its layer waits for its x
+// and for batch b-2's y to have left the slot, and its download runs while
+// batch b+1 computes.  Each batch is one whole-batch forward, so the weights
+// are streamed once per batch and y_host[b] equals moe_forward on x_host[b].
+int hostio_batches_impl(const moe_shape& s, int nb, const void* const* x_host, const void* Wg,
+                        const float* bias, const void* W1, const void* W3, const void* W2,
+                        void* const* y_host, void* ws, size_t ws_bytes, cudaStream_t st) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (nb < 1 || !x_host || !y_host) return MOE_ERR_INVALID_ARG;
+    for (int b = 0; b < nb; ++b)
+        if (!x_host[b] || !y_host[b]) return MOE_ERR_INVALID_ARG;
+    if (s.T == 0) return MOE_OK;
+    if (!ok_ptr(Wg) || !ok_opt(bias) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_hostio_batches_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
+    const size_t io_bytes = (size_t)s.T * s.d * 2;
+    const size_t slot = align_up(io_bytes, 256);
+    char* base = static_cast<char*>(ws) + moe_forward_workspace_bytes(s);
+    CopyStreams* cs = copy_streams();
+    if (!cs) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(cs->mu);
+    cudaEvent_t* ev = cs->evb;  // [0] start, [1+i] x in slot i, [3+i] slot i read, [5+i] y out, [7] end
+    bool ok = cudaEventRecord(ev[0], st) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->up, ev[0], 0) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->down, ev[0], 0) == cudaSuccess;
+    for (int b = 0; ok && b < nb; ++b) {
+        const int i = b & 1;
+        char* x_dev = base + (size_t)i * slot;
+        char* y_dev = base + (size_t)(2 + i) * slot;
+        if (b >= 2) ok = cudaStreamWaitEvent(cs->up, ev[3 + i], 0) == cudaSuccess;
+        ok = ok &&
+             cudaMemcpyAsync(x_dev, x_host[b], io_bytes, cudaMemcpyHostToDevice, cs->up) ==
+                 cudaSuccess &&
+             cudaEventRecord(ev[1 + i], cs->up) == cudaSuccess &&
+             cudaStreamWaitEvent(st, ev[1 + i], 0) == cudaSuccess;
+        if (ok && b >= 2) ok = cudaStreamWaitEvent(st, ev[5 + i], 0) == cudaSuccess;
+        FwdOptions opt;
+        opt.clear_status = b == 0;  // an expired wait in any batch stays reported
+        ok = ok &&
+             forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st,
+                          nullptr, opt) == MOE_OK &&
+             cudaEventRecord(ev[3 + i], st) == cudaSuccess &&
+             cudaStreamWaitEvent(cs->down, ev[3 + i], 0) == cudaSuccess &&
+             cudaMemcpyAsync(y_host[b], y_dev, io_bytes, cudaMemcpyDeviceToHost, cs->down) ==
+                 cudaSuccess &&
+             cudaEventRecord(ev[5 + i], cs->down) == cudaSuccess;
+    }
+    ok = ok && cudaEventRecord(ev[7], cs->down) == cudaSuccess &&
+         cudaStreamWaitEvent(st, ev[7], 0) == cudaSuccess;
+    return ok ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -338,6 +399,12 @@ size_t moe_forward_hostio_workspace_bytes(moe_shape s) {
     return fwd_layout(s).total + 2 * io;
 }
 
+size_t moe_forward_hostio_batches_workspace_bytes(moe_shape s) {
+    if (check_shape(s)) return 0;
+    const size_t io = align_up((size_t)s.T * s.d * 2, 256);
+    return fwd_layout(s).total + 4 * io;
+}
+
 int moe_route(moe_shape s, const void* x, const void* Wg, const float* bias, int32_t* idx,
               float* gate, float* logits, void* stream) {
     int rc = check_shape(s);
@@ -357,7 +424,7 @@ int moe_dispatch(moe_shape s, const int32_t* idx, const void* x, int32_t* offset
                     !ok_ptr(x_sorted)))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = launch_dispatch_index(s, idx, offsets, perm_tok, inv, nullptr, st);
+    rc = launch_dispatch_index(s, idx, offsets, perm_tok, inv, st);
     if (rc) return rc;
     return launch_dispatch_scatter(s, x, inv, x_sorted, st);
 }
@@ -493,6 +560,14 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
                        size_t ws_bytes, void* stream) {
     return hostio_impl(s, x_host, Wg, bias, W1, W3, W2, y_host, ws, ws_bytes,
                        static_cast<cudaStream_t>(stream), -1, -1, kDefaultWaitTimeoutNs);
+}
+
+int moe_forward_hostio_batches(moe_shape s, int n_batches, const void* const* x_host,
+                               const void* Wg, const float* bias, const void* W1,
+                               const void* W3, const void* W2, void* const* y_host, void* ws,
+                               size_t ws_bytes, void* stream) {
+    return hostio_batches_impl(s, n_batches, x_host, Wg, bias, W1, W3, W2, y_host, ws, ws_bytes,
+                               static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward_hostio_stall_test(moe_shape s, const void* x_host, const void* Wg,

@@ -61,7 +61,7 @@ __device__ __forceinline__ int ld_shared_cluster_s32(uint32_t addr) {
 __global__ void __launch_bounds__(kIndexThreads, 1)
     index_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                  int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
-                 int32_t* __restrict__ inv, int* status_to_clear) {
+                 int32_t* __restrict__ inv) {
     __shared__ int s_pos[kIndexWarps][kMaxExperts + 1];  // counts, then next positions
     __shared__ int s_total[kMaxExperts];                  // this CTA's rows per expert
     __shared__ int s_base[kMaxExperts];                   // first row of each expert in this CTA
@@ -71,7 +71,6 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
     const int rank = (int)sm100::cluster_ctarank();
     const int C = (int)cluster_size();
     grid_dependency_wait();
-    if (status_to_clear && tid == 0 && rank == 0) *status_to_clear = 0;
 
     const int n = T * k;
     const int nwarps = kIndexWarps * C;
@@ -208,8 +207,7 @@ __global__ void __launch_bounds__(256)
 }  // namespace dispatch
 
 int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offsets,
-                          int32_t* perm_tok, int32_t* inv, int* status_to_clear,
-                          cudaStream_t stream) {
+                          int32_t* perm_tok, int32_t* inv, cudaStream_t stream) {
     using namespace dispatch;
     if (s.E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
     // cluster size: enough CTAs for runs of about kSlotsPerWarp slots per warp
@@ -230,8 +228,8 @@ int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offse
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, index_kernel, idx, s.T, s.E, s.k, offsets, perm_tok, inv,
-                              status_to_clear) == cudaSuccess
+    return cudaLaunchKernelEx(&cfg, index_kernel, idx, s.T, s.E, s.k, offsets, perm_tok,
+                              inv) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

@@ -8,11 +8,9 @@
 
 namespace moe {
 
-// offsets [E+1], perm_tok [T*k], inv [T,k] from idx [T,k]; when status_to_clear
-// is non-null the kernel also zeroes that device status word.
+// offsets [E+1], perm_tok [T*k], inv [T,k] from idx [T,k].
 int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offsets,
-                          int32_t* perm_tok, int32_t* inv, int* status_to_clear,
-                          cudaStream_t stream);
+                          int32_t* perm_tok, int32_t* inv, cudaStream_t stream);
 
 // x_sorted[inv[t,s]] = x[t].
 int launch_dispatch_scatter(const moe_shape& s, const void* x, const int32_t* inv, void* x_sorted,

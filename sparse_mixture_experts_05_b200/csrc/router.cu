@@ -44,6 +44,7 @@
 #include <climits>
 
 #include "common.cuh"
+#include "expert_gemm.cuh"
 #include "router.cuh"
 #include "sm100.cuh"
 
@@ -122,23 +123,53 @@ __device__ __forceinline__ uint4 rms_scale8(const uint4& v, const uint4& gm, flo
 // 16-byte slot of row r (local to the CTA's staged range) of a W_r plane.
 __device__ __forceinline__ int w_slot(int r) { return r ^ (((r >> 3) & 3) << 1); }
 
+// Copies the W_r rows g0 + r0 .. g0 + r0 + nr - 1 of every 8-expert plane into
+// shared memory (plane nt starts plane_rows 16-byte rows after plane nt - 1;
+// local row r goes to slot w_slot(r)).  E a multiple of 8: 16-byte asynchronous
+// copies, waited for with cp_async_wait_all; otherwise plain stores (experts
+// past E read as zero).
+template <int NT>
+__device__ __forceinline__ void stage_wr(uint8_t* s_w, int plane_rows, int g0, int r0, int nr,
+                                         const uint16_t* __restrict__ wg, int E, int lane) {
+    if ((E & 7) == 0) {
+        const uint32_t a = sm100::smem_u32(s_w);
+        for (int i = lane; i < NT * nr; i += 32) {
+            const int nt = i / nr;
+            const int r = r0 + i - nt * nr;
+            cp_async_16(a + (uint32_t)((nt * plane_rows + w_slot(r)) * 16),
+                        wg + (int64_t)(g0 + r) * E + nt * 8);
+        }
+    } else {
+        for (int i = lane; i < NT * nr * 8; i += 32) {
+            const int j = i & 7;
+            const int rest = i >> 3;
+            const int nt = rest / nr;
+            const int r = r0 + rest - nt * nr;
+            const int n = nt * 8 + j;
+            const uint16_t v = n < E ? wg[(int64_t)(g0 + r) * E + n] : (uint16_t)0;
+            reinterpret_cast<uint16_t*>(s_w)[(nt * plane_rows + w_slot(r)) * 8 + j] = v;
+        }
+    }
+}
+
 __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
     return v > bv || (v == bv && id < bid) || bid == INT_MAX;
 }
 
 // Top-k of the logits v (fragment layout of the MMA accumulator: v[nt][i] is
-// token (i < 2 ? g : g + 8) of the tile, expert nt*8 + 2*t4 + (i & 1)), softmax
-// over the k, and the stores of idx, gate and (optionally) the logits.  Kept out
-// of line: it runs in one warp per tile, after the x loads' registers are dead.
+// token row0 + (i < 2 ? g : g + 8), expert nt*8 + 2*t4 + (i & 1)), softmax over
+// the k, and the stores of idx, gate and (optionally) the logits for the rows
+// below row_end.  Kept out of line: it runs in one warp per tile, after the x
+// loads' registers are dead.
 template <int NT>
-__device__ __noinline__ void select_and_store(float (&v)[NT][4], int tile, int T, int E, int k,
-                                              int g, int t4, int32_t* __restrict__ idx,
+__device__ __noinline__ void select_and_store(float (&v)[NT][4], int row0, int row_end, int E,
+                                              int k, int g, int t4, int32_t* __restrict__ idx,
                                               float* __restrict__ gate,
                                               float* __restrict__ logits) {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        const int row = tile * 16 + g + 8 * half;
-        const bool rv = row < T;
+        const int row = row0 + g + 8 * half;
+        const bool rv = row < row_end;
         if (logits && rv) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -220,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                   const float* __restrict__ bias, int T, int d, int E, int k, int C,
                   int32_t* __restrict__ idx, float* __restrict__ gate,
                   float* __restrict__ logits, const uint16_t* __restrict__ gamma, float eps,
-                  uint16_t* __restrict__ u_out) {
+                  uint16_t* __restrict__ u_out, int* __restrict__ status_to_clear) {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ float s_ss[kWarps][16];  // kNorm: per-warp sums of squares of the tile's rows
     // k blocks whose x loads are issued together (halved when normalising, which
@@ -239,34 +270,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t s_w = sm100::smem_u32(smem);
     const uint32_t s_part = s_w + (uint32_t)(NT * rows_cap * 16);
     grid_dependency_wait();
+    if (status_to_clear && blockIdx.x == 0 && tid == 0) *status_to_clear = 0;
 
     const int q = rank * kWarps + warp;          // this warp's k range
     const int kb_lo = (q * nkb) / KS;
     const int kb_hi = ((q + 1) * nkb) / KS;
     // Each warp stages the W_r rows of its own k range, plane by plane (8
     // experts per plane), so it waits only for its own copies (no block barrier).
-    {
-        const int r0 = (kb_lo - cta_kb0) * 32;
-        const int nr = (kb_hi - kb_lo) * 32;
-        if ((E & 7) == 0) {
-            for (int i = lane; i < NT * nr; i += 32) {
-                const int nt = i / nr;
-                const int r = r0 + i - nt * nr;
-                cp_async_16(s_w + (uint32_t)((nt * rows_cap + w_slot(r)) * 16),
-                            wg + (int64_t)(cta_kb0 * 32 + r) * E + nt * 8);
-            }
-        } else {
-            for (int i = lane; i < NT * nr * 8; i += 32) {
-                const int j = i & 7;
-                const int rest = i >> 3;
-                const int nt = rest / nr;
-                const int r = r0 + rest - nt * nr;
-                const int n = nt * 8 + j;
-                const uint16_t v = n < E ? wg[(int64_t)(cta_kb0 * 32 + r) * E + n] : (uint16_t)0;
-                reinterpret_cast<uint16_t*>(smem)[(nt * rows_cap + w_slot(r)) * 8 + j] = v;
-            }
-        }
-    }
+    stage_wr<NT>(smem, rows_cap, cta_kb0 * 32, (kb_lo - cta_kb0) * 32, (kb_hi - kb_lo) * 32, wg,
+                 E, lane);
 
     // ldmatrix: lane supplies row i = lane & 7 of matrix m = lane >> 3, i.e. row
     // 8 (i >> 1) + 2 m + (i & 1) of the k block
@@ -438,12 +450,266 @@ __global__ void __launch_bounds__(kThreads, 2)
                         if (n < E) v[nt][i] = __fadd_rn(v[nt][i], bias[n]);
                     }
             }
-            select_and_store<NT>(v, tile, T, E, k, g, t4, idx, gate, logits);
+            select_and_store<NT>(v, tile * 16, min(T, tile * 16 + 16), E, k, g, t4, idx, gate,
+                                 logits);
         }
     }
     cp_async_wait_all();
     // no CTA leaves while the reducing warp may still read its partial sums
     sm100::cluster_sync_all();
+}
+
+// ---------------------------------------------------------------------------
+// Streaming kernel for batches with at least one 16-token tile per SM (where
+// the cluster kernel runs at C = 1).  One CTA per SM, and the tokens are cut
+// into tiles of hrows = ceil(T / (waves * CTAs)) <= 16 rows, so every SM reads
+// nearly the same number of rows (16-row tiles left a third of the SMs with
+// half the work at T = 4096).  A producer warp streams each tile's eight k
+// ranges into a ring of shared-memory slots with TMA, one copy per slot: x is
+// viewed in 3-D as [T rows][d / 64 chunks][64 columns], and a box of hrows rows
+// by nbox = min(8, d / 512) chunks lands as hrows rows of nbox * 128 bytes
+// (128-byte swizzle; rows past T read as zeros).  Small copies cost: the same
+// bytes as 14-row boxes of one chunk each, eight copies per slot, ran slower
+// than the cluster kernel.  Consumer warp q owns k range q of every tile, as warp q of the cluster
+// kernel does at C = 1: the same W_r staging, the same A fragments (read from
+// the swizzled slot instead of global memory), the same MMAs in the same k
+// order and the same left-to-right sum over the ranges, so both kernels give a
+// token the same bits.  Each consumer warp has its own ring of depth slots,
+// so consecutive uses of a slot belong to one warp, which has consumed use u - 1
+// before it waits for use u: with one ring shared by all warps, a warp that had
+// run ahead could wait for use u of a slot whose use u - 1 had not landed yet,
+// and the parity wait passed on the phase before.  The ranges' partial sums of a
+// tile go to one of two shared-memory buffers, and an epilogue warp adds them,
+// adds the bias and selects the top k while the consumers go on to the next
+// tile (mbarriers in both directions; with the selection inside a loop bound by
+// a per-tile barrier, a rotating warp doing it, the kernel ran no faster than
+// the cluster kernel).  Every mbarrier wait is bounded; an expired one is
+// recorded in the workspace status word (when given, with where it gave up in
+// the words after it) and the kernel runs on to its end.
+namespace stream {
+constexpr int kConsumers = kWarps;             // warps 0-7: one per k range
+constexpr int kProducer = kConsumers;          // warp 8: TMA
+constexpr int kThreads = (kConsumers + 2) * 32;  // warp 9: sums, top k, stores
+constexpr int kMaxDepth = 4;                   // ring slots per consumer warp
+constexpr int kRowsMax = 16;                   // a slot holds up to 16 rows
+constexpr int kBoxesPerStage = 8;              // chunks of 64 columns per slot at most
+constexpr int kSmemLimit = 227 * 1024;
+}  // namespace stream
+
+struct StreamParams {
+    const uint16_t* wg;
+    const float* bias;
+    int T, d, E, k;
+    int hrows;       // rows per token tile (<= 16)
+    int ntiles;      // ceil(T / hrows)
+    int rb;          // 64-column chunks per k range (d / 512)
+    int nbox;        // chunks per slot, min(8, rb); rb is a multiple of it
+    int nch;         // ring stages per k range (rb / nbox)
+    int depth;       // ring slots per consumer warp (slots = 8 * depth)
+    int slot_bytes;  // kRowsMax * nbox * 128
+    int32_t* idx;
+    float* gate;
+    float* logits;
+    int* status;     // workspace status word (nullable)
+    int clear;       // zero *status before anything else
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// First expired wait of the launch: status word 1 = which wait (1 producer on a
+// free slot, 2 consumer on a full slot, 3 consumer on a free partial buffer,
+// 4 epilogue on a written partial buffer), word 2 = the stage or tile index,
+// word 3 = the CTA, word 4 = the barrier's parity waited for.
+__device__ __noinline__ void note_expired(int* status, int kind, int index, int parity) {
+    if (status && atomicCAS(status + 1, 0, kind) == 0) {
+        status[2] = index;
+        status[3] = (int)blockIdx.x;
+        status[4] = parity;
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(stream::kThreads, 1)
+    router_stream_kernel(const __grid_constant__ CUtensorMap tmx, const StreamParams p) {
+    using namespace stream;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = sm100::smem_u32(smem_raw);
+    const uint32_t s_x = (raw + 1023u) & ~1023u;  // 128-byte swizzle wants 1024-byte rows of 8
+    uint8_t* smem = smem_raw + (s_x - raw);
+    const int nslots = kConsumers * p.depth;
+    uint8_t* s_wp = smem + nslots * p.slot_bytes;
+    const uint32_t s_w = sm100::smem_u32(s_wp);
+    float4* s_part = reinterpret_cast<float4*>(s_wp + NT * p.d * 16);
+    uint64_t* full = reinterpret_cast<uint64_t*>(s_part + 2 * kConsumers * 32 * NT);
+    uint64_t* empty = full + nslots;
+    uint64_t* pfull = empty + nslots;  // [2] a tile's partial sums written (one per consumer warp)
+    uint64_t* pempty = pfull + 2;      // [2] a tile's partial sums read (the epilogue warp)
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nslots; ++i) {
+            sm100::mbar_init(&full[i], 1);
+            sm100::mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            sm100::mbar_init(&pfull[i], kConsumers);
+            sm100::mbar_init(&pempty[i], 1);
+        }
+        sm100::fence_barrier_init();
+    }
+    if (warp == kProducer && lane == 0) sm100::tma_prefetch_map(&tmx);
+    __syncthreads();
+    grid_dependency_wait();
+    if (p.clear && p.status && blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0;
+    bool ok = true;
+
+    if (warp == kProducer) {
+        // stage n of consumer q (n = local tile * nch + chunk) goes to slot
+        // q * depth + n % depth, its use n / depth; issued tile by tile, range by range
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
+                const int row0 = tile * p.hrows;
+                for (int q = 0; q < kConsumers; ++q) {
+                    for (int c = 0; c < p.nch; ++c) {
+                        const int n = it * p.nch + c;
+                        const int slot = q * p.depth + n % p.depth;
+                        const int use = n / p.depth;
+                        if (use > 0 && !sm100::mbar_wait(&empty[slot], (use - 1) & 1, p.timeout_ns)) {
+                            ok = false;
+                            note_expired(p.status, 1, n, (use - 1) & 1);
+                        }
+                        sm100::mbar_arrive_expect_tx(&full[slot],
+                                                     (uint32_t)(p.nbox * p.hrows * 128));
+                        sm100::tma_load_3d(smem + slot * p.slot_bytes, &tmx, &full[slot], 0,
+                                           q * p.rb + c * p.nbox, row0);
+                    }
+                }
+            }
+        }
+    } else if (warp < kConsumers) {
+        const int q = warp;  // this warp's k range
+        const int g = lane >> 2;
+        const int t4 = lane & 3;
+        const int range_kb = (p.d >> 5) / kConsumers;
+        const int kb_lo = q * range_kb;
+        stage_wr<NT>(s_wp, p.d, 0, kb_lo * 32, range_kb * 32, p.wg, p.E, lane);
+        const int lrow = 8 * ((lane & 7) >> 1) + 2 * (lane >> 3) + (lane & 1);
+        const uint32_t lane_off = (uint32_t)(w_slot(lrow) * 16);
+        // lane (g, t4) reads 8 columns t4*8.. of a 32-column k block from rows g and
+        // g + 8 of a slot: row r, chunk b is the 128-byte line r * nbox + b of the
+        // slot, whose 16-byte piece u the swizzle moves to u ^ (line & 7); rows g
+        // and g + 8 share that key (8 * nbox lines apart)
+        const uint32_t pitch = (uint32_t)(p.nbox * 128);
+        const uint32_t row_g = (uint32_t)g * pitch, row_g8 = (uint32_t)(g + 8) * pitch;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
+            float c[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
+            for (int cc = 0; cc < p.nch; ++cc) {
+                const int n = it * p.nch + cc;
+                const int slot = q * p.depth + n % p.depth;
+                const int par = (n / p.depth) & 1;
+                if (!sm100::mbar_wait(&full[slot], par, p.timeout_ns)) {
+                    ok = false;
+                    note_expired(p.status, 2, n, par);
+                }
+                if (it == 0 && cc == 0) {  // this warp's W_r rows must have landed
+                    cp_async_wait_all();
+                    __syncwarp();
+                }
+                const uint32_t sx = s_x + (uint32_t)(slot * p.slot_bytes);
+                const int kb0 = kb_lo + cc * p.nbox * 2;
+                for (int b = 0; b < p.nbox; ++b) {
+                    const uint32_t box = sx + (uint32_t)(b * 128);
+                    const int key = (g * p.nbox + b) & 7;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t ch = (uint32_t)(((hh * 4 + t4) ^ key) * 16);
+                        const uint4 a0 = ld_shared_v4(box + row_g + ch);
+                        const uint4 a1 = ld_shared_v4(box + row_g8 + ch);
+                        const uint32_t blk =
+                            s_w + (uint32_t)((kb0 + b * 2 + hh) * 32 * 16) + lane_off;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            uint32_t bf[4];
+                            ldmatrix_x4_trans(blk + (uint32_t)(nt * p.d * 16), bf);
+                            mma_bf16_16816(c[nt], a0.x, a1.x, a0.y, a1.y, bf[0], bf[1]);
+                            mma_bf16_16816(c[nt], a0.z, a1.z, a0.w, a1.w, bf[2], bf[3]);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(&empty[slot]);
+            }
+            // partial sums into buffer it & 1, once the epilogue has read what
+            // tile it - 2 left there
+            const int pb = it & 1;
+            if (it >= 2 && !sm100::mbar_wait(&pempty[pb], ((it >> 1) - 1) & 1, p.timeout_ns)) {
+                ok = false;
+                note_expired(p.status, 3, it, ((it >> 1) - 1) & 1);
+            }
+            float4* mine = s_part + ((pb * kConsumers + q) * 32 + lane) * NT;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mine[nt] = make_float4(c[nt][0], c[nt][1], c[nt][2], c[nt][3]);
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&pfull[pb]);
+        }
+        cp_async_wait_all();  // (a warp without tiles still waits for its W_r copies)
+    } else {
+        // epilogue: the ranges' partial sums of each tile added left to right
+        const int g = lane >> 2;
+        const int t4 = lane & 3;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
+            const int pb = it & 1;
+            if (!sm100::mbar_wait(&pfull[pb], (it >> 1) & 1, p.timeout_ns)) {
+                ok = false;
+                note_expired(p.status, 4, it, (it >> 1) & 1);
+            }
+            float v[NT][4];
+            const float4* part = s_part + (pb * kConsumers * 32 + lane) * NT;
+#pragma unroll
+            for (int w = 0; w < kConsumers; ++w)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float4 pv = part[w * 32 * NT + nt];
+                    if (w == 0) {
+                        v[nt][0] = pv.x; v[nt][1] = pv.y; v[nt][2] = pv.z; v[nt][3] = pv.w;
+                    } else {
+                        v[nt][0] = __fadd_rn(v[nt][0], pv.x);
+                        v[nt][1] = __fadd_rn(v[nt][1], pv.y);
+                        v[nt][2] = __fadd_rn(v[nt][2], pv.z);
+                        v[nt][3] = __fadd_rn(v[nt][3], pv.w);
+                    }
+                }
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&pempty[pb]);  // free for tile it + 2
+            if (p.bias) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = nt * 8 + 2 * t4 + (i & 1);
+                        if (n < p.E) v[nt][i] = __fadd_rn(v[nt][i], p.bias[n]);
+                    }
+            }
+            const int row0 = tile * p.hrows;
+            select_and_store<NT>(v, row0, min(p.T, row0 + p.hrows), p.E, p.k, g, t4, p.idx,
+                                 p.gate, p.logits);
+        }
+    }
+    if (!ok) record_error(p.status, kDeviceTimeoutBase | kRoleRouter);
 }
 
 }  // namespace router
@@ -460,17 +726,104 @@ int router_cluster(const moe_shape& s) {
     return C;
 }
 
+namespace {
+
+// Launch plan of the streaming kernel, or false where the cluster kernel runs:
+// C > 1, fewer 16-token tiles than SMs, d not a multiple of 512 (a k range must
+// be whole 64-column chunks, and up to 8 of them or a multiple of 8), or W_r plus
+// eight ring slots over the shared memory.
+struct StreamPlan {
+    int ctas, hrows, ntiles, rb, nbox, nch, depth, slot_bytes;
+    size_t smem;
+};
+
+bool stream_plan(const moe_shape& s, int C, StreamPlan& pl) {
+    using namespace router::stream;
+    const int NT = (s.E + 7) / 8;
+    if (C != 1 || s.d % 512 != 0) return false;
+    const int sms = device_sm_count();
+    const int t16 = (s.T + 15) / 16;
+    if (sms <= 0 || t16 < sms) return false;
+    const int waves = (t16 + sms - 1) / sms;
+    pl.ctas = sms;
+    pl.hrows = (s.T + waves * sms - 1) / (waves * sms);
+    pl.ntiles = (s.T + pl.hrows - 1) / pl.hrows;
+    pl.rb = s.d / 512;
+    pl.nbox = std::min(kBoxesPerStage, pl.rb);
+    if (pl.rb % pl.nbox != 0) return false;
+    pl.nch = pl.rb / pl.nbox;
+    pl.slot_bytes = kRowsMax * pl.nbox * 128;
+    // alignment slack, W_r planes, two buffers of partial sums and their four
+    // mbarriers; each slot also takes two mbarriers; at least one slot per warp
+    const size_t fixed = 1024 + (size_t)NT * s.d * 16 +
+                         (size_t)2 * kConsumers * 32 * NT * sizeof(float4) + 4 * sizeof(uint64_t);
+    if (fixed >= (size_t)kSmemLimit) return false;
+    const size_t per_warp_slot = (size_t)kConsumers * (pl.slot_bytes + 16);
+    pl.depth = (int)std::min<size_t>(kMaxDepth, ((size_t)kSmemLimit - fixed) / per_warp_slot);
+    if (pl.depth < 1) return false;
+    pl.smem = fixed + (size_t)pl.depth * per_warp_slot;
+    return true;
+}
+
+}  // namespace
+
 int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                   int32_t* idx, float* gate, float* logits, cudaStream_t stream, int cluster,
-                  const RouterNorm* norm) {
+                  const RouterNorm* norm, int* status, bool clear_status) {
     using namespace router;
     if (s.T == 0) return MOE_OK;
     const int NT = (s.E + 7) / 8;
     // The cluster size fixes the order in which the partial sums of a logit are
     // added; a caller that runs one batch in token chunks passes the size chosen
-    // for the whole batch so every chunk rounds the same way.
+    // for the whole batch so every chunk rounds the same way (both kernels add
+    // them in the same order at C = 1).
     const int C = cluster <= 0 ? router_cluster(s) : cluster;
     if (C != 1 && C != 2 && C != 4 && C != 8) return MOE_ERR_INVALID_ARG;
+    int* to_clear = clear_status ? status : nullptr;
+    StreamPlan pl;
+    if (!norm && stream_plan(s, C, pl)) {
+        // x as [T][d / 64][64]: box of hrows rows by nbox 64-column chunks
+        CUtensorMap tmx;
+        const uint64_t dims[3] = {64, (uint64_t)s.d / 64, (uint64_t)s.T};
+        const uint64_t strides[2] = {128, (uint64_t)s.d * 2};
+        const uint32_t box[3] = {64, (uint32_t)pl.nbox, (uint32_t)pl.hrows};
+        if (!make_bf16_map_3d(&tmx, x, dims, strides, box)) return MOE_ERR_CUDA;
+        StreamParams p;
+        p.wg = static_cast<const uint16_t*>(Wg);
+        p.bias = bias;
+        p.T = s.T;
+        p.d = s.d;
+        p.E = s.E;
+        p.k = s.k;
+        p.hrows = pl.hrows;
+        p.ntiles = pl.ntiles;
+        p.rb = pl.rb;
+        p.nbox = pl.nbox;
+        p.nch = pl.nch;
+        p.depth = pl.depth;
+        p.slot_bytes = pl.slot_bytes;
+        p.idx = idx;
+        p.gate = gate;
+        p.logits = logits;
+        p.status = status;
+        p.clear = clear_status ? 1 : 0;
+        p.timeout_ns = kDefaultWaitTimeoutNs;
+        auto run_stream = [&](auto kern) {
+            if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)pl.smem))
+                return MOE_ERR_CUDA;
+            return launch_pdl(kern, dim3(pl.ctas), dim3(stream::kThreads), pl.smem, stream, tmx,
+                              p) == cudaSuccess
+                       ? MOE_OK
+                       : MOE_ERR_CUDA;
+        };
+        switch (NT) {
+            case 1: return run_stream(router_stream_kernel<1>);
+            case 2: return run_stream(router_stream_kernel<2>);
+            case 3: return run_stream(router_stream_kernel<3>);
+            case 4: return run_stream(router_stream_kernel<4>);
+            default: return MOE_ERR_UNSUPPORTED;
+        }
+    }
     const int nkb = s.d / 32;
     const int rows_cap = ((nkb + C - 1) / C) * 32;
     const size_t smem = (size_t)NT * rows_cap * 16 + (size_t)2 * kWarps * 32 * NT * 16;
@@ -500,7 +853,7 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, kern, xp, wp, bias, s.T, s.d, s.E, s.k, C, idx, gate,
-                                  logits, gp, eps, up) == cudaSuccess
+                                  logits, gp, eps, up, to_clear) == cudaSuccess
                    ? MOE_OK
                    : MOE_ERR_CUDA;
     };

@@ -21,9 +21,13 @@ struct RouterNorm {
     void* u;            // [T, d] bf16 (out)
 };
 
+// status: the workspace status word (nullable); with clear_status the router
+// zeroes it first (it is the first kernel of a forward), and an expired
+// bounded wait of the streaming kernel is recorded there.
 int launch_router(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                   int32_t* idx, float* gate, float* logits, cudaStream_t stream, int cluster = 0,
-                  const RouterNorm* norm = nullptr);
+                  const RouterNorm* norm = nullptr, int* status = nullptr,
+                  bool clear_status = false);
 
 // The cluster size launch_router picks for shape s (depends on T, d and the SM count).
 int router_cluster(const moe_shape& s);

@@ -188,3 +188,26 @@ def test_empty_batch_is_a_no_op_on_host():
     S = binding.MoeShape(0, 128, 256, 8, 2)
     for fn, nargs in (("moe_route", 7), ("moe_combine", 5)):
         assert _call(fn, S, *([None] * nargs)) == moe.MOE_OK
+
+
+def test_hostio_batches_rejects_bad_arguments_on_host():
+    S = binding.MoeShape(64, 128, 256, 8, 2)
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    arr = (P * 2)(1 << 20, 1 << 21)
+    holey = (P * 2)(1 << 20, None)
+    big = ctypes.c_size_t(1 << 30)
+    fn = "moe_forward_hostio_batches"
+    assert _call(fn, S, 0, arr, good, None, good, good, good, arr, good, big, None) == \
+        moe.MOE_ERR_INVALID_ARG                                         # no batches
+    assert _call(fn, S, 2, None, good, None, good, good, good, arr, good, big, None) == \
+        moe.MOE_ERR_INVALID_ARG                                         # no x array
+    assert _call(fn, S, 2, arr, good, None, good, good, good, holey, good, big, None) == \
+        moe.MOE_ERR_INVALID_ARG                                         # a null y entry
+    need = moe.moe_forward_hostio_batches_workspace_bytes((64, 128, 256, 8, 2))
+    assert need == moe.moe_forward_workspace_bytes((64, 128, 256, 8, 2)) + 4 * 64 * 128 * 2
+    assert _call(fn, S, 2, arr, good, None, good, good, good, arr, good,
+                 ctypes.c_size_t(need - 1), None) == moe.MOE_ERR_WORKSPACE
+    # T = 0 enqueues nothing
+    assert _call(fn, binding.MoeShape(0, 128, 256, 8, 2), 2, arr, None, None, None, None, None,
+                 arr, None, ctypes.c_size_t(0), None) == moe.MOE_OK

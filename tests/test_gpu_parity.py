@@ -284,6 +284,34 @@ def test_hostio_token_chunks_equal_the_whole_batch(T):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
 
 
+@pytest.mark.parametrize("T,n", [(700, 5), (64, 1), (2048, 3)],
+                         ids=["five-batches", "one-batch", "three-large-batches"])
+def test_hostio_batches_equal_per_batch_forwards(T, n):
+    """A queue of batches through two staging slots: batch b+1's upload and
+    batch b-1's download overlap batch b's layer.  Every batch must equal
+    moe_forward on its own x bit for bit (a slot reused before its previous
+    batch's download or layer finished would show here), and the call twice on
+    the same workspace must order itself after the first."""
+    d = 1024
+    inp = make_inputs(T, d, 512, 8, 2, seed=61, bias=True)
+    dev = to_dev(inp)
+    shape = inp["shape"]
+    args = (dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    g = torch.Generator().manual_seed(62)
+    xs = [(inp["x"].float() * (1.0 + 0.25 * b) +
+           0.1 * torch.randn(T, d, generator=g)).to(torch.bfloat16) for b in range(n)]
+    refs = [moe.moe_forward(shape, x.cuda(), *args).cpu() for x in xs]
+    xs_host = [x.pin_memory() for x in xs]
+    ys_host = [torch.full((T, d), 5.0, dtype=torch.bfloat16).pin_memory() for _ in range(n)]
+    ws = moe.workspace(moe.moe_forward_hostio_batches_workspace_bytes(shape), "cuda")
+    for _ in range(2):
+        moe.moe_forward_hostio_batches(shape, xs_host, *args, ys_host, ws)
+    torch.cuda.synchronize()
+    for b in range(n):
+        assert torch.equal(ys_host[b], refs[b]), f"batch {b}"
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+
+
 @pytest.mark.parametrize("T,stall_chunk", [(2048, 0), (2048, 1), (2048, 2), (300, 0)],
                          ids=["first-of-three-chunks", "middle-chunk", "last-chunk", "one-chunk"])
 def test_hostio_reports_a_timeout_in_any_chunk(T, stall_chunk):
