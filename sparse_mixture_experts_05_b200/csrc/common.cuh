@@ -17,7 +17,6 @@ constexpr int kRoleProducer = 1;
 constexpr int kRoleMma = 2;
 constexpr int kRoleEpilogue = 3;
 constexpr int kRoleTest = 4;
-constexpr int kRoleRouter = 5;
 
 // Default bound on any device-side wait: far above the longest legitimate wait
 // (one tile of the longest contraction, tens of microseconds).

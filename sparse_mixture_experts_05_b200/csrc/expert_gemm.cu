@@ -1151,18 +1151,4 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
                   : launch<false>(mh, m2, m2, oo, p2, t2, stream);
 }
 
-bool make_bf16_map_3d(CUtensorMap* map, const void* base, const uint64_t (&dims)[3],
-                      const uint64_t (&strides)[2], const uint32_t (&box)[3]) {
-    gemm::EncodeTiledFn fn = gemm::encode_fn();
-    if (!fn) return false;
-    cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-    cuuint64_t st[2] = {strides[0], strides[1]};
-    cuuint32_t bx[3] = {box[0], box[1], box[2]};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), d, st, bx,
-                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 }  // namespace moe

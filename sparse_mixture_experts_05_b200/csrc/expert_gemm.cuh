@@ -1,7 +1,6 @@
 // expert_gemm.cuh -- host entry of the grouped expert GEMMs (expert_gemm.cu).
 #pragma once
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -21,10 +20,5 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
                  uint64_t timeout_ns, int stall_after, cudaStream_t stream,
                  void* mid_event, const float* b1 = nullptr, const float* b3 = nullptr,
                  const float* b2 = nullptr);
-
-// 3-D bf16 tensor map (dims innermost first, strides in bytes of dims 1 and 2),
-// 128-byte swizzle, coordinates past a dimension read as zeros.
-bool make_bf16_map_3d(CUtensorMap* map, const void* base, const uint64_t (&dims)[3],
-                      const uint64_t (&strides)[2], const uint32_t (&box)[3]);
 
 }  // namespace moe

@@ -44,12 +44,14 @@
 #include <climits>
 
 #include "common.cuh"
-#include "expert_gemm.cuh"
 #include "router.cuh"
 #include "sm100.cuh"
+#include "tma_map.cuh"
 
 namespace moe {
 namespace router {
+
+constexpr int kRoleRouter = 5;  // status role of the streaming kernel's waits
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
