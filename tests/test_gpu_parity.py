@@ -78,6 +78,35 @@ def test_route_wide_rows(T, d, E, k):
     check_routing(idx.cpu().numpy(), gate.cpu().numpy(), o_idx, o_gate, o_logits, k)
 
 
+# Batches with at least one 16-token tile per SM run the streaming router (one
+# CTA per SM, a TMA ring per consumer warp, an epilogue warp); these shapes
+# cover its variants on 148 SMs: the threshold batch (148 tiles of 16 rows),
+# ragged last tiles, E not a multiple of 8 (W_r staged with plain stores), two
+# and four 8-expert planes, rings 1 to 4 slots deep holding 2 to 8 chunks of 64
+# columns, with the router bias and the logits output.
+STREAM_ROUTE = {
+    "threshold-d4096": (2368, 4096, 8, 2),
+    "ragged-E5k3-d1024": (3001, 1024, 5, 3),
+    "E32k8-d1024": (4097, 1024, 32, 8),
+    "E16k4-d2048": (5000, 2048, 16, 4),
+    "d1536": (2500, 1536, 8, 2),
+}
+
+
+@pytest.mark.parametrize("name", list(STREAM_ROUTE))
+def test_route_streaming_kernel_shapes(name):
+    T, d, E, k = STREAM_ROUTE[name]
+    inp = make_inputs(T, d, 128, E, k, seed=30 + E + k, bias=True)
+    dev = to_dev(inp)
+    idx, gate, logits = moe.moe_route(inp["shape"], dev["x"], dev["Wg"], dev["bias"],
+                                      want_logits=True)
+    torch.cuda.synchronize()
+    o_idx, o_gate, o_logits = oracle.route(inp["x"], inp["Wg"], E, k, bias=inp["bias"])
+    lerr = np.max(np.abs(logits.cpu().numpy() - o_logits))
+    assert lerr < 1e-4, lerr
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), o_idx, o_gate, o_logits, k)
+
+
 def test_route_ties_to_lower_index():
     inp = make_inputs(48, 128, 256, 8, 2, seed=12)
     inp["Wg"][:, 6] = inp["Wg"][:, 3]
@@ -279,6 +308,27 @@ def test_hostio_token_chunks_equal_the_whole_batch(T):
     ws = moe.workspace(moe.moe_forward_hostio_workspace_bytes(inp["shape"]), "cuda")
     for _ in range(2):  # twice on the same buffers: the pipeline orders itself after earlier work
         moe.moe_forward_hostio(inp["shape"], x_host, *args, y_host, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y_dev.cpu(), y_host)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+
+
+@pytest.mark.parametrize("T,E,k", [(3200, 5, 3), (4097, 32, 8), (3500, 16, 4)],
+                         ids=["E5k3", "E32k8", "E16k4"])
+def test_hostio_chunks_route_alike_in_both_router_kernels(T, E, k):
+    """The host-I/O pipeline routes its small edge chunks through the cluster
+    router (C = 1, the whole batch's split) and its large middle chunk through
+    the streaming router; the whole batch, through moe_forward, takes the
+    streaming router for every token.  Equal y bit for bit means both kernels
+    gave every token the same expert ids and the same gate bits."""
+    inp = make_inputs(T, 1024, 256, E, k, seed=40 + E, bias=True)
+    dev = to_dev(inp)
+    args = (dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    y_dev = moe.moe_forward(inp["shape"], dev["x"], *args)
+    x_host = inp["x"].clone().pin_memory()
+    y_host = torch.full((T, 1024), 3.0, dtype=torch.bfloat16).pin_memory()
+    ws = moe.workspace(moe.moe_forward_hostio_workspace_bytes(inp["shape"]), "cuda")
+    moe.moe_forward_hostio(inp["shape"], x_host, *args, y_host, ws)
     torch.cuda.synchronize()
     assert torch.equal(y_dev.cpu(), y_host)
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
