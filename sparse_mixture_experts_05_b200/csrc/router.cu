@@ -515,6 +515,9 @@ struct StreamParams {
     int* status;     // workspace status word (nullable)
     int clear;       // zero *status before anything else
     uint64_t timeout_ns;
+    const uint16_t* gamma;  // RMSNorm_2 weights [d] (norm mode)
+    float eps;
+    uint16_t* u_out;        // u [T, d] (norm mode)
 };
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -538,7 +541,20 @@ __device__ __noinline__ void note_expired(int* status, int kind, int index, int 
     }
 }
 
-template <int NT>
+// Barrier 1 among the consumer warps only (norm mode: the row sums of squares of
+// a tile meet before any warp scales its range).
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(stream::kConsumers * 32) : "memory");
+}
+
+// kNorm: the block edge's RMSNorm_2 as in router_kernel's norm mode, from the
+// tile already in shared memory (one stage per k range, nch == 1): pass A adds
+// the squares of the warp's range per row (in k order, then over the quad),
+// the eight ranges' sums meet after one consumer barrier and are added in range
+// order, and pass B scales the same shared-memory rows, stores u and feeds the
+// MMAs -- the same operations in the same order as the cluster kernel, so u and
+// the routing have the same bits in both.
+template <int NT, bool kNorm>
 __global__ void __launch_bounds__(stream::kThreads, 1)
     router_stream_kernel(const __grid_constant__ CUtensorMap tmx, const StreamParams p) {
     using namespace stream;
@@ -550,7 +566,8 @@ __global__ void __launch_bounds__(stream::kThreads, 1)
     uint8_t* s_wp = smem + nslots * p.slot_bytes;
     const uint32_t s_w = sm100::smem_u32(s_wp);
     float4* s_part = reinterpret_cast<float4*>(s_wp + NT * p.d * 16);
-    uint64_t* full = reinterpret_cast<uint64_t*>(s_part + 2 * kConsumers * 32 * NT);
+    float* s_ss = reinterpret_cast<float*>(s_part + 2 * kConsumers * 32 * NT);  // [2][8][16]
+    uint64_t* full = reinterpret_cast<uint64_t*>(s_ss + 2 * kConsumers * 16);
     uint64_t* empty = full + nslots;
     uint64_t* pfull = empty + nslots;  // [2] a tile's partial sums written (one per consumer warp)
     uint64_t* pempty = pfull + 2;      // [2] a tile's partial sums read (the epilogue warp)
@@ -631,16 +648,65 @@ __global__ void __launch_bounds__(stream::kThreads, 1)
                 }
                 const uint32_t sx = s_x + (uint32_t)(slot * p.slot_bytes);
                 const int kb0 = kb_lo + cc * p.nbox * 2;
+                float inv0 = 1.0f, inv1 = 1.0f;
+                if constexpr (kNorm) {
+                    // pass A: this warp's range of rows g and g + 8
+                    float ss0 = 0.0f, ss1 = 0.0f;
+                    for (int b = 0; b < p.nbox; ++b) {
+                        const uint32_t box = sx + (uint32_t)(b * 128);
+                        const int key = (g * p.nbox + b) & 7;
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t ch = (uint32_t)(((hh * 4 + t4) ^ key) * 16);
+                            ss0 = sum_squares8(ld_shared_v4(box + row_g + ch), ss0);
+                            ss1 = sum_squares8(ld_shared_v4(box + row_g8 + ch), ss1);
+                        }
+                    }
+                    ss0 = __fadd_rn(ss0, __shfl_xor_sync(0xffffffffu, ss0, 1));
+                    ss0 = __fadd_rn(ss0, __shfl_xor_sync(0xffffffffu, ss0, 2));
+                    ss1 = __fadd_rn(ss1, __shfl_xor_sync(0xffffffffu, ss1, 1));
+                    ss1 = __fadd_rn(ss1, __shfl_xor_sync(0xffffffffu, ss1, 2));
+                    float* my_ss = s_ss + ((it & 1) * kConsumers + q) * 16;
+                    if (t4 == 0) {
+                        my_ss[g] = ss0;
+                        my_ss[g + 8] = ss1;
+                    }
+                    // the buffer alternates per tile: a warp reads buffer it & 1
+                    // before it reaches the next tile's barrier, which every
+                    // writer of that buffer passes before writing it again
+                    consumers_sync();
+                    const float* all_ss = s_ss + (it & 1) * kConsumers * 16;
+                    float tot0 = all_ss[g], tot1 = all_ss[g + 8];
+#pragma unroll
+                    for (int w = 1; w < kConsumers; ++w) {
+                        tot0 = __fadd_rn(tot0, all_ss[w * 16 + g]);
+                        tot1 = __fadd_rn(tot1, all_ss[w * 16 + g + 8]);
+                    }
+                    inv0 = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot0, (float)p.d), p.eps)));
+                    inv1 = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot1, (float)p.d), p.eps)));
+                }
+                const int r0 = tile * p.hrows + g;
+                const bool u0 = kNorm && g < p.hrows && r0 < p.T;
+                const bool u1 = kNorm && g + 8 < p.hrows && r0 + 8 < p.T;
                 for (int b = 0; b < p.nbox; ++b) {
                     const uint32_t box = sx + (uint32_t)(b * 128);
                     const int key = (g * p.nbox + b) & 7;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const uint32_t ch = (uint32_t)(((hh * 4 + t4) ^ key) * 16);
-                        const uint4 a0 = ld_shared_v4(box + row_g + ch);
-                        const uint4 a1 = ld_shared_v4(box + row_g8 + ch);
-                        const uint32_t blk =
-                            s_w + (uint32_t)((kb0 + b * 2 + hh) * 32 * 16) + lane_off;
+                        uint4 a0 = ld_shared_v4(box + row_g + ch);
+                        uint4 a1 = ld_shared_v4(box + row_g8 + ch);
+                        const int kb = kb0 + b * 2 + hh;
+                        if constexpr (kNorm) {
+                            // pass B: u = bf16((U * inv) * gamma), stored for the scatter
+                            const uint4 gm = __ldg(reinterpret_cast<const uint4*>(p.gamma) + kb * 4 + t4);
+                            a0 = rms_scale8(a0, gm, inv0);
+                            a1 = rms_scale8(a1, gm, inv1);
+                            uint4* urow = reinterpret_cast<uint4*>(p.u_out) + kb * 4 + t4;
+                            if (u0) urow[(int64_t)r0 * (p.d / 8)] = a0;
+                            if (u1) urow[(int64_t)(r0 + 8) * (p.d / 8)] = a1;
+                        }
+                        const uint32_t blk = s_w + (uint32_t)(kb * 32 * 16) + lane_off;
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             uint32_t bf[4];
@@ -732,14 +798,15 @@ namespace {
 
 // Launch plan of the streaming kernel, or false where the cluster kernel runs:
 // C > 1, fewer 16-token tiles than SMs, d not a multiple of 512 (a k range must
-// be whole 64-column chunks, and up to 8 of them or a multiple of 8), or W_r plus
-// eight ring slots over the shared memory.
+// be whole 64-column chunks, and up to 8 of them or a multiple of 8), W_r plus
+// eight ring slots over the shared memory, or (norm mode) a k range of more than
+// one slot.
 struct StreamPlan {
     int ctas, hrows, ntiles, rb, nbox, nch, depth, slot_bytes;
     size_t smem;
 };
 
-bool stream_plan(const moe_shape& s, int C, StreamPlan& pl) {
+bool stream_plan(const moe_shape& s, int C, bool norm, StreamPlan& pl) {
     using namespace router::stream;
     const int NT = (s.E + 7) / 8;
     if (C != 1 || s.d % 512 != 0) return false;
@@ -754,11 +821,14 @@ bool stream_plan(const moe_shape& s, int C, StreamPlan& pl) {
     pl.nbox = std::min(kBoxesPerStage, pl.rb);
     if (pl.rb % pl.nbox != 0) return false;
     pl.nch = pl.rb / pl.nbox;
+    if (norm && pl.nch != 1) return false;
     pl.slot_bytes = kRowsMax * pl.nbox * 128;
-    // alignment slack, W_r planes, two buffers of partial sums and their four
-    // mbarriers; each slot also takes two mbarriers; at least one slot per warp
+    // alignment slack, W_r planes, two buffers of partial sums, two of row sums
+    // of squares, four mbarriers; each slot also takes two mbarriers; at least
+    // one slot per warp
     const size_t fixed = 1024 + (size_t)NT * s.d * 16 +
-                         (size_t)2 * kConsumers * 32 * NT * sizeof(float4) + 4 * sizeof(uint64_t);
+                         (size_t)2 * kConsumers * 32 * NT * sizeof(float4) +
+                         (size_t)2 * kConsumers * 16 * sizeof(float) + 4 * sizeof(uint64_t);
     if (fixed >= (size_t)kSmemLimit) return false;
     const size_t per_warp_slot = (size_t)kConsumers * (pl.slot_bytes + 16);
     pl.depth = (int)std::min<size_t>(kMaxDepth, ((size_t)kSmemLimit - fixed) / per_warp_slot);
@@ -783,7 +853,7 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
     if (C != 1 && C != 2 && C != 4 && C != 8) return MOE_ERR_INVALID_ARG;
     int* to_clear = clear_status ? status : nullptr;
     StreamPlan pl;
-    if (!norm && stream_plan(s, C, pl)) {
+    if (stream_plan(s, C, norm != nullptr, pl)) {
         // x as [T][d / 64][64]: box of hrows rows by nbox 64-column chunks
         CUtensorMap tmx;
         const uint64_t dims[3] = {64, (uint64_t)s.d / 64, (uint64_t)s.T};
@@ -810,6 +880,9 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
         p.status = status;
         p.clear = clear_status ? 1 : 0;
         p.timeout_ns = kDefaultWaitTimeoutNs;
+        p.gamma = norm ? static_cast<const uint16_t*>(norm->gamma) : nullptr;
+        p.eps = norm ? norm->eps : 0.0f;
+        p.u_out = norm ? static_cast<uint16_t*>(norm->u) : nullptr;
         auto run_stream = [&](auto kern) {
             if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)pl.smem))
                 return MOE_ERR_CUDA;
@@ -818,13 +891,18 @@ int launch_router(const moe_shape& s, const void* x, const void* Wg, const float
                        ? MOE_OK
                        : MOE_ERR_CUDA;
         };
+#define MOE_STREAM_CASE(N)                                                              \
+    case N:                                                                             \
+        return norm ? run_stream(router_stream_kernel<N, true>)                         \
+                    : run_stream(router_stream_kernel<N, false>);
         switch (NT) {
-            case 1: return run_stream(router_stream_kernel<1>);
-            case 2: return run_stream(router_stream_kernel<2>);
-            case 3: return run_stream(router_stream_kernel<3>);
-            case 4: return run_stream(router_stream_kernel<4>);
+            MOE_STREAM_CASE(1)
+            MOE_STREAM_CASE(2)
+            MOE_STREAM_CASE(3)
+            MOE_STREAM_CASE(4)
             default: return MOE_ERR_UNSUPPORTED;
         }
+#undef MOE_STREAM_CASE
     }
     const int nkb = s.d / 32;
     const int rows_cap = ((nkb + C - 1) / C) * 32;

@@ -29,10 +29,15 @@ BLOCK_CASES = {
     "ragged": (77, 256, 384, 8, 2, 5, True),
     "decode-d4096": (16, 4096, 256, 8, 2, 6, False),
     "mid-d2048": (300, 2048, 256, 8, 2, 7, True),
+    # at least one 16-token tile per SM (148 SMs): the streaming router, which
+    # normalises the tile it holds in shared memory
+    "stream-d1024": (3000, 1024, 512, 8, 2, 11, True),
+    "stream-d4096": (2400, 4096, 256, 8, 2, 12, False),
 }
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "quarter", "decode-d4096", "mid-d2048"])
+@pytest.mark.parametrize("name", ["tiny", "ragged", "quarter", "decode-d4096", "mid-d2048",
+                                  "stream-d1024", "stream-d4096"])
 def test_block_forward_matches_oracle(name):
     if name in BLOCK_CASES:
         T, d, d_ff, E, k, seed, bias = BLOCK_CASES[name]
@@ -67,7 +72,7 @@ def test_block_zero_down_projection_returns_the_residual_exactly():
     assert torch.equal(H, dev["x"])
 
 
-@pytest.mark.parametrize("name", ["quarter", "decode-d4096"])
+@pytest.mark.parametrize("name", ["quarter", "decode-d4096", "stream-d1024", "stream-d4096"])
 def test_router_normalised_rows_match_oracle_rmsnorm(name):
     """The router writes u = bf16((U * inv) * gamma) into the block workspace (right
     after moe_forward's part) for the scatter; u equals the oracle's RMSNorm to
@@ -92,3 +97,4 @@ def test_router_normalised_rows_match_oracle_rmsnorm(name):
     diff = np.abs(uv - u_ref)
     assert np.all(diff <= bf16_ulp(u_ref) * 1.0001 + 1e-30)
     assert np.mean(diff > 0) < 1e-3
+
