@@ -570,9 +570,11 @@ def _omp_threads(n):
 
 
 def oracle_per_config():
-    """The oracle's full forward (expert-major loop, fp64) on the tiny and
-    quarter-width workloads, on all host cores and on one core (quarter on one
-    core: a 64-token sample through the per-token loop); about 10 s in all."""
+    """The oracle's full forward (expert-major loop, fp64) on the tiny,
+    quarter-width and decode workloads on all host cores, and on one core (the
+    quarter-width and decode ones on a sample through the per-token loop: 64 and
+    4 tokens); about 15 s in all.  The prefill and skewed batches are timed on a
+    token sample only (`cpu_baseline` itself): their full forward takes minutes."""
     import numpy as np
 
     import oracle
@@ -580,12 +582,13 @@ def oracle_per_config():
     oracle.build()
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     out = {}
-    for name in ("tiny", "quarter"):
+    one_core_sample = {"tiny": None, "quarter": 64, "decode": 4}
+    for name in ("tiny", "quarter", "decode"):
         inp = workload_inputs(name)
         T, d, d_ff, E, k = inp["shape"]
         args = (inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k)
         runs = [("all_cores", cores, None)]
-        runs.append(("one_core", 1, None if name == "tiny" else 64))
+        runs.append(("one_core", 1, one_core_sample[name]))
         for label, threads, sample in runs:
             if not _omp_threads(threads):
                 continue
