@@ -98,3 +98,52 @@ def test_router_normalised_rows_match_oracle_rmsnorm(name):
     assert np.all(diff <= bf16_ulp(u_ref) * 1.0001 + 1e-30)
     assert np.mean(diff > 0) < 1e-3
 
+
+
+def test_block_forward_prefill_size_sampled_tokens():
+    """The block edges at the Mixtral 8x7B prefill size (T = 4096, d = 4096,
+    d_ff = 14336), where the streaming router normalises the rows it holds in
+    shared memory: u on every row against the oracle's RMSNorm (within one
+    bf16 ulp), and H on at least 256 sampled tokens -- the first and last row of
+    every expert group, the near ties, random ones -- against U plus the
+    oracle's layer on the GPU's u (so both sides route the same rows; near ties
+    of the k-th place are counted and left out, as for the layer's own parity)."""
+    inp = workload_inputs("prefill")
+    T, d, d_ff, E, k = inp["shape"]
+    gamma = _gamma(d, 15)
+    dev = to_dev(inp)
+    ws = moe.workspace(moe.moe_block_workspace_bytes(inp["shape"]), "cuda")
+    H = moe.moe_block_forward(inp["shape"], dev["x"], gamma.cuda(), dev["Wg"], None, dev["W1"],
+                              dev["W3"], dev["W2"], eps=1e-5, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    off = moe.moe_forward_workspace_bytes(inp["shape"])
+    u = ws[off:off + T * d * 2].view(torch.bfloat16).view(T, d).cpu()
+    u_ref = oracle.bf16_to_f64(oracle.rmsnorm(inp["x"], gamma, 1e-5))
+    diff = np.abs(bf16_values(u) - u_ref)
+    assert np.all(diff <= bf16_ulp(u_ref) * 1.0001 + 1e-30)
+    assert np.mean(diff > 0) < 1e-3
+
+    o_idx, _, o_logits = oracle.route(u, inp["Wg"], E, k)
+    kth_tie, _ = oracle.near_tie_flags(o_logits, k)
+    off_e, perm, _ = oracle.dispatch(o_idx, E)
+    picks = {0, T - 1}
+    for e in range(E):
+        if off_e[e + 1] > off_e[e]:
+            picks.update([int(perm[off_e[e]]), int(perm[off_e[e + 1] - 1])])
+    picks.update(np.nonzero(kth_tie)[0].tolist())
+    rng = np.random.default_rng(29)
+    rest = np.setdiff1d(np.arange(T), np.fromiter(picks, int))
+    picks.update(rng.choice(rest, max(0, 256 - len(picks)), replace=False).tolist())
+    toks = np.array(sorted(picks))
+    y_ref, _, _ = oracle.forward_tokens(toks, u, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k)
+    keep = ~kth_tie[toks]
+    U = bf16_values(inp["x"][torch.from_numpy(toks).long()])
+    H_ref = U + y_ref
+    Hv = bf16_values(H[torch.from_numpy(toks).long().cuda()])
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    err = np.abs(Hv - H_ref)[keep]
+    bound = (0.5 * bf16_ulp(H_ref) + Y_TOL * rms)[keep]
+    assert np.all(err <= bound), float(np.max(err / bound))
+    print("tokens", len(toks), "near ties left out", int((~keep).sum()),
+          "max err / bound", float(np.max(err / bound)))

@@ -15,8 +15,8 @@ from _parity import to_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("T,d,d_ff", [(64, 128, 256), (700, 256, 512)],
-                         ids=["single-cta", "cta-pair"])
+@pytest.mark.parametrize("T,d,d_ff", [(64, 128, 256), (700, 256, 512), (2600, 1024, 256)],
+                         ids=["single-cta", "cta-pair", "streaming-router"])
 def test_forward_replays_in_a_cuda_graph(T, d, d_ff):
     inp = make_inputs(T, d, d_ff, 8, 2, seed=70, bias=True)
     shape = inp["shape"]
