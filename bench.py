@@ -697,10 +697,10 @@ def run_ours(a):
         "tflops_layer": round(alg["flops_total"] / (max_ms / 1000) / 1e12, 1),
         "bracket_ms_incl_flush": round(bracket_ms, 3),
     }
-    if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
-        line["extras"] = extras_loop(ctx, a.steps, device, local)
     if a.workload in ("prefill", "skew") and not a.no_secondary:
         line["router_isolated"] = router_isolated(ctx, device)
+    if a.workload == "prefill" and not a.no_secondary and a.tokens is None and a.experts is None:
+        line["extras"] = extras_loop(ctx, a.steps, device, local)
     del ctx
     torch.cuda.empty_cache()
 
