@@ -321,8 +321,10 @@ def extras_loop(ctx, steps, device, local):
     the plain layer so that all see the same clocks and power state (L2 flushed
     before every call, nvidia-smi sampled throughout): the block with its edges,
     the layer with expert biases, and the load-balancing term on the router's
-    logits.  Reports each one's mean time and its difference from the plain
-    layer measured in the same loop."""
+    logits.  Reports each one's mean time, and its difference from the plain
+    layer as the median over the steps of the two calls' difference within a
+    step (neighbouring calls see the same clock, which drifts as the GPU heats),
+    over at least 30 steps."""
     import torch
 
     import sparse_mixture_experts_05_b200 as moe
@@ -363,7 +365,7 @@ def extras_loop(ctx, steps, device, local):
     times = {name: [] for name in calls}
     clock = ClockSampler(local)
     clock.start()
-    for i in range(steps):
+    for i in range(max(steps, 30)):
         for name, call in calls.items():
             ctx["flush"].fill_(i & 0xFF)
             e0 = torch.cuda.Event(enable_timing=True)
@@ -377,14 +379,19 @@ def extras_loop(ctx, steps, device, local):
     if moe.moe_read_device_status(ws_b) != moe.MOE_OK:
         raise RuntimeError("device status error in the block forward")
     out = {name: round(statistics.mean(v), 4) for name, v in times.items()}
-    out["block_minus_plain_on_u_ms"] = round(out["block_forward_ms"] - out["plain_on_u_ms"], 4)
-    out["bias_minus_plain_ms"] = round(out["forward_bias_ms"] - out["plain_ms"], 4)
+
+    def paired(a, b):
+        return round(statistics.median(x - y for x, y in zip(times[a], times[b])), 4)
+    out["block_minus_plain_on_u_ms"] = paired("block_forward_ms", "plain_on_u_ms")
+    out["bias_minus_plain_ms"] = paired("forward_bias_ms", "plain_ms")
+    out["steps"] = len(times["plain_ms"])
     out["clocks"] = clocks
     out["note"] = ("same batch, calls interleaved step by step (plain, plain on u, block, bias, "
                    "aux); block = RMSNorm inside the router + layer + residual in the combine, "
-                   "gamma ~ 1 + N(0, 0.04); plain on u = the layer on the block's own "
+                   "gamma ~ 1 + 0.2 N(0, 1); plain on u = the layer on the block's own "
                    "normalised rows (same routing and GEMM tiles as the block); bias = expert "
-                   "Linear biases b1, b3, b2; aux = load-balancing term over the T x E logits")
+                   "Linear biases b1, b3, b2; aux = load-balancing term over the T x E logits; "
+                   "*_minus_* = median over the steps of the difference within a step")
     return out
 
 
