@@ -321,10 +321,13 @@ def extras_loop(ctx, steps, device, local):
     the plain layer so that all see the same clocks and power state (L2 flushed
     before every call, nvidia-smi sampled throughout): the block with its edges,
     the layer with expert biases, and the load-balancing term on the router's
-    logits.  Reports each one's mean time, and its difference from the plain
-    layer as the median over the steps of the two calls' difference within a
-    step (neighbouring calls see the same clock, which drifts as the GPU heats),
-    over at least 30 steps."""
+    logits.  The order of the five calls rotates by one every step, so each
+    call runs in each place equally often over whole rotations (at least 30
+    steps) and no call always follows the same one.  Reports each one's mean
+    time and
+    its difference from the plain layer as the mean over the steps of the two
+    calls' difference within a step (calls of one step see the same clock,
+    which drifts as the GPU heats)."""
     import torch
 
     import sparse_mixture_experts_05_b200 as moe
@@ -365,8 +368,12 @@ def extras_loop(ctx, steps, device, local):
     times = {name: [] for name in calls}
     clock = ClockSampler(local)
     clock.start()
-    for i in range(max(steps, 30)):
-        for name, call in calls.items():
+    names = list(calls)
+    n_steps = -(-max(steps, 30) // len(names)) * len(names)
+    for i in range(n_steps):
+        for j in range(len(names)):
+            name = names[(i + j) % len(names)]
+            call = calls[name]
             ctx["flush"].fill_(i & 0xFF)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
@@ -381,7 +388,7 @@ def extras_loop(ctx, steps, device, local):
     out = {name: round(statistics.mean(v), 4) for name, v in times.items()}
 
     def paired(a, b):
-        return round(statistics.median(x - y for x, y in zip(times[a], times[b])), 4)
+        return round(statistics.mean(x - y for x, y in zip(times[a], times[b])), 4)
     out["block_minus_plain_on_u_ms"] = paired("block_forward_ms", "plain_on_u_ms")
     out["bias_minus_plain_ms"] = paired("forward_bias_ms", "plain_ms")
     out["steps"] = len(times["plain_ms"])
@@ -391,8 +398,50 @@ def extras_loop(ctx, steps, device, local):
                    "gamma ~ 1 + 0.2 N(0, 1); plain on u = the layer on the block's own "
                    "normalised rows (same routing and GEMM tiles as the block); bias = expert "
                    "Linear biases b1, b3, b2; aux = load-balancing term over the T x E logits; "
-                   "*_minus_* = median over the steps of the difference within a step")
+                   "order rotated every step; *_minus_* = mean over the steps of the "
+                   "difference within a step")
     return out
+
+
+def graph_step_ms(ctx, steps):
+    """The step replayed from a CUDA graph of one moe_forward (captured once),
+    the L2 flushed before each replay, each replay between two events with the
+    host waiting for it: the device time of the layer without the host's
+    per-launch work, which the eager steps of a sub-0.1 ms workload can carry
+    (the host issues each eager step's six launches through the Python binding
+    while the device waits).  Returns (median, mean) in ms."""
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    inp = ctx["inp"]
+    shape = ctx["shape"]
+    args = tuple(inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        moe.moe_forward(shape, *args, y=ctx["y"], ws=ctx["ws"])
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        moe.moe_forward(shape, *args, y=ctx["y"], ws=ctx["ws"])
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms = []
+    for i in range(steps):
+        ctx["flush"].fill_(i & 0xFF)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    if moe.moe_read_device_status(ctx["ws"]) != moe.MOE_OK:
+        raise RuntimeError("device status error in the graph replays")
+    del graph
+    return statistics.median(ms), statistics.mean(ms)
 
 
 def secondary_workload(name, steps, warmup, device, rank, local, pg, peaks):
@@ -416,6 +465,14 @@ def secondary_workload(name, steps, warmup, device, rank, local, pg, peaks):
            "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
            "ms_per_step_profiled": round(pmean, 4), "expert_rows": ctx["counts"],
            "clocks": clocks}
+    if name in ("decode", "quarter", "tiny"):
+        g_med, g_mean = graph_step_ms(ctx, w_steps)
+        g_med = reduce_max(pg, g_med, device)
+        out["graph"] = {"ms_per_step_median": round(g_med, 4),
+                        "ms_per_step_mean": round(g_mean, 4),
+                        "tokens_per_s": round(T * world / (g_med / 1e3), 1),
+                        "how": "the same step replayed from a CUDA graph of moe_forward, host "
+                               "waiting for each replay (device time without host launch work)"}
     if name == "decode":
         gbs = alg["bytes_experts_decode"] / (gemm / 1000) / 1e9
         out.update({"experts_gbs": round(gbs, 1),
