@@ -68,6 +68,10 @@ def parse(argv=None):
     ap.add_argument("--vs-cublas", action="store_true",
                     help="instead of the step: time the expert GEMMs against cuBLAS batched "
                          "bf16 GEMMs of the same shapes (equal rows per expert), alternating")
+    ap.add_argument("--block-vs-plain", action="store_true",
+                    help="instead of the step: the block forward (RMSNorm inside the router, "
+                         "residual in the combine) and the plain layer on the block's own "
+                         "normalised rows, alternating (a short run for profiler launch lists)")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -923,12 +927,60 @@ def vs_cublas(a):
         "clocks": clocks}))
 
 
+def block_vs_plain(a):
+    """The block forward and the plain layer on the block's normalised rows u,
+    alternating step by step on the workload's batch (L2 flushed before each
+    call), W warm-up pairs then K timed pairs; prints one JSON line of the
+    per-call CUDA-event times.  Same routing and GEMM tiles on both sides, so
+    the difference is the block edges' cost."""
+    import torch
+
+    import sparse_mixture_experts_05_b200 as moe
+    device = "cuda:0"
+    torch.cuda.set_device(0)
+    ctx = time_workload(a.workload, 1, 3, device, 0, a.tokens, a.experts)
+    inp = ctx["inp"]
+    shape = ctx["shape"]
+    T, d = shape[0], shape[1]
+    x, Wg, bias, W1, W3, W2 = (inp[key] for key in ("x", "Wg", "bias", "W1", "W3", "W2"))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(5)
+    gamma = (1 + 0.2 * torch.randn(d, generator=gen, device=device)).to(torch.bfloat16)
+    ws_b = moe.workspace(moe.moe_block_workspace_bytes(shape), device)
+    H = torch.empty(T, d, dtype=torch.bfloat16, device=device)
+    moe.moe_block_forward(shape, x, gamma, Wg, bias, W1, W3, W2, H=H, ws=ws_b)
+    off = moe.moe_forward_workspace_bytes(shape)
+    u = ws_b[off:off + T * d * 2].view(torch.bfloat16).view(T, d).clone()
+    calls = {"plain_on_u_ms": lambda: moe.moe_forward(shape, u, Wg, bias, W1, W3, W2,
+                                                      y=ctx["y"], ws=ctx["ws"]),
+             "block_forward_ms": lambda: moe.moe_block_forward(shape, x, gamma, Wg, bias, W1, W3,
+                                                               W2, H=H, ws=ws_b)}
+    times = {name: [] for name in calls}
+    for i in range(a.warmup + a.steps):
+        for name, call in calls.items():
+            ctx["flush"].fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            e1.synchronize()
+            if i >= a.warmup:
+                times[name].append(e0.elapsed_time(e1))
+    if moe.moe_read_device_status(ws_b) != moe.MOE_OK:
+        raise RuntimeError("device status error in the block forward")
+    print(json.dumps({"workload": WORKLOAD_NAMES[a.workload], "steps": a.steps,
+                      **{name: [round(t, 4) for t in v] for name, v in times.items()}}))
+
+
 def main(argv=None):
     a = parse(argv)
     if a.impl == "reference":
         run_reference(a)
     elif a.vs_cublas:
         vs_cublas(a)
+    elif a.block_vs_plain:
+        block_vs_plain(a)
     else:
         run_ours(a)
     return 0
