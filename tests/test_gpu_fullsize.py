@@ -150,3 +150,28 @@ def test_expert_sampled_rows(case):
                                     bf16_values(xs_sub), row_expert, inp["W1"], inp["W3"],
                                     inp["W2"], h_ref, o_ref)
     print(name, "h elements differing from the oracle", frac, "o error / bound", worst)
+
+
+def test_hostio_batches_prefill_size_bit_exact():
+    """The queue of host batches at the Mixtral prefill size (the bench's
+    end-to-end path): three batches of 4096 tokens, two of them with the same
+    host buffers (pinned) and one pageable, each equal to moe_forward on its x
+    bit for bit."""
+    inp = workload_inputs("prefill")
+    dev = to_dev(inp)
+    T, d, d_ff, E, k = inp["shape"]
+    args = (dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    g = torch.Generator().manual_seed(81)
+    x1 = inp["x"].clone()
+    x2 = (inp["x"].float() + 0.5 * torch.randn(T, d, generator=g)).to(torch.bfloat16)
+    refs = [moe.moe_forward(inp["shape"], x.cuda(), *args).cpu() for x in (x1, x2)]
+    xs = [x1.pin_memory(), x2.pin_memory(), x1.clone()]          # the last one pageable
+    ys = [torch.empty(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    ys.append(torch.empty(T, d, dtype=torch.bfloat16))
+    ws = moe.workspace(moe.moe_forward_hostio_batches_workspace_bytes(inp["shape"]), "cuda")
+    moe.moe_forward_hostio_batches(inp["shape"], xs, *args, ys, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    assert torch.equal(ys[0], refs[0])
+    assert torch.equal(ys[1], refs[1])
+    assert torch.equal(ys[2], refs[0])
