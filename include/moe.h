@@ -23,7 +23,8 @@
  *        W2       [E, d_ff, d]  bf16   down projection
  *        y        [T, d]        bf16   layer output
  *  - Every pointer except `stream` is DEVICE memory owned by the caller, except
- *    in moe_forward_hostio where x and y are HOST memory.  The library never
+ *    in the host-I/O entry points (moe_forward_hostio, moe_forward_hostio_batches
+ *    and their test hooks) where x and y are HOST memory.  The library never
  *    allocates or frees memory and never synchronises, except
  *    moe_read_device_status (documented there).  All work is enqueued
  *    asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream)
@@ -271,6 +272,24 @@ int moe_forward_hostio_batches(moe_shape s, int n_batches, const void* const* x_
                                const void* Wg, const float* bias, const void* W1,
                                const void* W3, const void* W2, void* const* y_host, void* ws,
                                size_t ws_bytes, void* stream);
+
+/*
+ * moe_forward_hostio_batches_stall_test -- test hook for the error path of the
+ * queue of batches (no counterpart on the pages).  Runs
+ * moe_forward_hostio_batches with the expert kernels' TMA producer of batch
+ * `stall_batch` (0 = first; past the last stalls nothing) stopping after
+ * `stall_after` (>= 0) pipeline stages, and that batch's device waits bounded
+ * by `timeout_ns` (1e3 .. 2e9).  The status word is cleared once, before the
+ * first batch, so moe_read_device_status(ws) reports MOE_ERR_DEVICE_TIMEOUT
+ * whichever batch's wait expired; that batch's y is incomplete, the others'
+ * are right, and the CUDA context stays usable.
+ */
+int moe_forward_hostio_batches_stall_test(moe_shape s, int n_batches,
+                                          const void* const* x_host, const void* Wg,
+                                          const float* bias, const void* W1, const void* W3,
+                                          const void* W2, void* const* y_host, void* ws,
+                                          size_t ws_bytes, int stall_batch, int stall_after,
+                                          uint64_t timeout_ns, void* stream);
 
 /*
  * moe_forward_hostio_stall_test -- test hook for the error path of the chunked

@@ -11,7 +11,8 @@ from .binding import (  # noqa: F401
     moe_block_workspace_bytes, moe_check_shape, moe_combine, moe_dispatch, moe_expert_swiglu,
     moe_expert_swiglu_bias, moe_expert_swiglu_stall_test, moe_expert_workspace_bytes, moe_forward,
     moe_forward_bias, moe_forward_hostio, moe_forward_hostio_batches,
-    moe_forward_hostio_batches_workspace_bytes, moe_forward_hostio_stall_test,
+    moe_forward_hostio_batches_stall_test, moe_forward_hostio_batches_workspace_bytes,
+    moe_forward_hostio_stall_test,
     moe_forward_hostio_workspace_bytes,
     moe_forward_profiled, moe_forward_static, moe_forward_workspace_bytes,
     moe_read_device_status, moe_route, status_string, workspace,

@@ -31,6 +31,7 @@ EXPORTS = (
     "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_bias", "moe_expert_swiglu_stall_test",
     "moe_combine", "moe_forward", "moe_forward_bias", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_hostio_stall_test",
     "moe_forward_hostio_batches_workspace_bytes", "moe_forward_hostio_batches",
+    "moe_forward_hostio_batches_stall_test",
     "moe_forward_static",
     "moe_aux_loss", "moe_block_workspace_bytes", "moe_block_forward", "moe_read_device_status",
 )
@@ -96,6 +97,9 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_hostio.argtypes = [S, P, P, P, P, P, P, P, P, Z, P]
         L.moe_forward_hostio_batches.restype = I
         L.moe_forward_hostio_batches.argtypes = [S, I, P, P, P, P, P, P, P, P, Z, P]
+        L.moe_forward_hostio_batches_stall_test.restype = I
+        L.moe_forward_hostio_batches_stall_test.argtypes = [S, I, P, P, P, P, P, P, P, P, Z, I,
+                                                            I, ctypes.c_uint64, P]
         L.moe_forward_hostio_stall_test.restype = I
         L.moe_forward_hostio_stall_test.argtypes = [S, P, P, P, P, P, P, P, P, Z, I, I,
                                                     ctypes.c_uint64, P]
@@ -406,6 +410,44 @@ def moe_forward_hostio_batches(shape, xs_host, Wg, bias, W1, W3, W2, ys_host, ws
                                             _p(Wg), _p(bias), _p(W1), _p(W3), _p(W2),
                                             ctypes.cast(yp, ctypes.c_void_p), _p(ws), ws.numel(),
                                             _stream(stream)))
+    return ys_host
+
+
+def _host_batches(shape, xs_host, ys_host):
+    T, d, d_ff, E, k = shape
+    if len(xs_host) != len(ys_host) or len(xs_host) < 1:
+        raise ValueError("xs_host and ys_host must be non-empty and of equal length")
+    for name, seq in (("xs_host", xs_host), ("ys_host", ys_host)):
+        for t in seq:
+            if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() \
+                    or tuple(t.shape) != (T, d):
+                raise ValueError(f"every {name} entry must be a contiguous CPU bf16 tensor "
+                                 f"of shape {(T, d)}")
+    n = len(xs_host)
+    xp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in xs_host])
+    yp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in ys_host])
+    return n, xp, yp
+
+
+def moe_forward_hostio_batches_stall_test(shape, xs_host, Wg, bias, W1, W3, W2, ys_host, ws,
+                                          stall_batch: int, stall_after: int, timeout_ns: int,
+                                          stream=None):
+    """moe_forward_hostio_batches with the expert producer of batch `stall_batch`
+    stopping after `stall_after` stages and that batch's waits bounded by
+    `timeout_ns` (test of the error path of the queue)."""
+    T, d, d_ff, E, k = shape
+    n, xp, yp = _host_batches(shape, xs_host, ys_host)
+    _dev(Wg, "Wg", torch.bfloat16, (d, E))
+    _dev(bias, "bias", torch.float32, (E,))
+    _dev(W1, "W1", torch.bfloat16, (E, d, d_ff))
+    _dev(W3, "W3", torch.bfloat16, (E, d, d_ff))
+    _dev(W2, "W2", torch.bfloat16, (E, d_ff, d))
+    _dev(ws, "ws", torch.uint8)
+    _check("moe_forward_hostio_batches_stall_test",
+           lib().moe_forward_hostio_batches_stall_test(
+               _shape(shape), n, ctypes.cast(xp, ctypes.c_void_p), _p(Wg), _p(bias), _p(W1),
+               _p(W3), _p(W2), ctypes.cast(yp, ctypes.c_void_p), _p(ws), ws.numel(),
+               int(stall_batch), int(stall_after), int(timeout_ns), _stream(stream)))
     return ys_host
 
 

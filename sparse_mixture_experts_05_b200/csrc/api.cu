@@ -310,7 +310,9 @@ int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const fl
 // are streamed once per batch and y_host[b] equals moe_forward on x_host[b].
 int hostio_batches_impl(const moe_shape& s, int nb, const void* const* x_host, const void* Wg,
                         const float* bias, const void* W1, const void* W3, const void* W2,
-                        void* const* y_host, void* ws, size_t ws_bytes, cudaStream_t st) {
+                        void* const* y_host, void* ws, size_t ws_bytes, cudaStream_t st,
+                        int stall_batch = -1, int stall_after = -1,
+                        uint64_t timeout_ns = kDefaultWaitTimeoutNs) {
     int rc = check_shape(s);
     if (rc) return rc;
     if (nb < 1 || !x_host || !y_host) return MOE_ERR_INVALID_ARG;
@@ -343,6 +345,10 @@ int hostio_batches_impl(const moe_shape& s, int nb, const void* const* x_host, c
         if (ok && b >= 2) ok = cudaStreamWaitEvent(st, ev[5 + i], 0) == cudaSuccess;
         FwdOptions opt;
         opt.clear_status = b == 0;  // an expired wait in any batch stays reported
+        if (b == stall_batch) {
+            opt.stall_after = stall_after;
+            opt.timeout_ns = timeout_ns;
+        }
         ok = ok &&
              forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st,
                           nullptr, opt) == MOE_OK &&
@@ -568,6 +574,19 @@ int moe_forward_hostio_batches(moe_shape s, int n_batches, const void* const* x_
                                size_t ws_bytes, void* stream) {
     return hostio_batches_impl(s, n_batches, x_host, Wg, bias, W1, W3, W2, y_host, ws, ws_bytes,
                                static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_hostio_batches_stall_test(moe_shape s, int n_batches,
+                                          const void* const* x_host, const void* Wg,
+                                          const float* bias, const void* W1, const void* W3,
+                                          const void* W2, void* const* y_host, void* ws,
+                                          size_t ws_bytes, int stall_batch, int stall_after,
+                                          uint64_t timeout_ns, void* stream) {
+    if (stall_batch < 0 || stall_after < 0) return MOE_ERR_INVALID_ARG;
+    if (timeout_ns < 1000 || timeout_ns > kDefaultWaitTimeoutNs) return MOE_ERR_INVALID_ARG;
+    return hostio_batches_impl(s, n_batches, x_host, Wg, bias, W1, W3, W2, y_host, ws, ws_bytes,
+                               static_cast<cudaStream_t>(stream), stall_batch, stall_after,
+                               timeout_ns);
 }
 
 int moe_forward_hostio_stall_test(moe_shape s, const void* x_host, const void* Wg,

@@ -211,3 +211,21 @@ def test_hostio_batches_rejects_bad_arguments_on_host():
     # T = 0 enqueues nothing
     assert _call(fn, binding.MoeShape(0, 128, 256, 8, 2), 2, arr, None, None, None, None, None,
                  arr, None, ctypes.c_size_t(0), None) == moe.MOE_OK
+
+
+def test_hostio_batches_stall_hook_rejects_bad_arguments_on_host():
+    S = binding.MoeShape(64, 128, 256, 8, 2)
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    arr = (P * 2)(1 << 20, 1 << 21)
+    big = ctypes.c_size_t(1 << 30)
+    t = ctypes.c_uint64(10 ** 6)
+    fn = "moe_forward_hostio_batches_stall_test"
+    assert _call(fn, S, 2, arr, good, None, good, good, good, arr, good, big, -1, 1, t,
+                 None) == moe.MOE_ERR_INVALID_ARG                          # negative batch
+    assert _call(fn, S, 2, arr, good, None, good, good, good, arr, good, big, 0, -1, t,
+                 None) == moe.MOE_ERR_INVALID_ARG                          # negative stage count
+    assert _call(fn, S, 2, arr, good, None, good, good, good, arr, good, big, 0, 1,
+                 ctypes.c_uint64(10), None) == moe.MOE_ERR_INVALID_ARG     # timeout too short
+    assert _call(fn, S, 0, arr, good, None, good, good, good, arr, good, big, 0, 1, t,
+                 None) == moe.MOE_ERR_INVALID_ARG                          # no batches

@@ -362,6 +362,37 @@ def test_hostio_batches_equal_per_batch_forwards(T, n):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
 
 
+@pytest.mark.parametrize("stall_batch", [0, 1, 2], ids=["first", "middle", "last"])
+def test_hostio_batches_report_a_timeout_in_any_batch(stall_batch):
+    """A queue of three batches on one workspace; the status word is cleared
+    once, before the first, so an expired wait in any batch must still read
+    MOE_ERR_DEVICE_TIMEOUT after the call, the other batches must be right, and a
+    normal call afterwards on the same workspace must report MOE_OK."""
+    T, d = 600, 256
+    inp = make_inputs(T, d, 256, 8, 2, seed=47, bias=True)
+    dev = to_dev(inp)
+    shape = inp["shape"]
+    args = (dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    g = torch.Generator().manual_seed(48)
+    xs = [(inp["x"].float() + 0.3 * b * torch.randn(T, d, generator=g)).to(torch.bfloat16)
+          for b in range(3)]
+    refs = [moe.moe_forward(shape, x.cuda(), *args).cpu() for x in xs]
+    xs_host = [x.pin_memory() for x in xs]
+    ys_host = [torch.zeros(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    ws = moe.workspace(moe.moe_forward_hostio_batches_workspace_bytes(shape), "cuda")
+    moe.moe_forward_hostio_batches_stall_test(shape, xs_host, *args, ys_host, ws,
+                                              stall_batch=stall_batch, stall_after=1,
+                                              timeout_ns=2_000_000)
+    assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    for b in range(3):
+        if b != stall_batch:
+            assert torch.equal(ys_host[b], refs[b]), f"batch {b}"
+    moe.moe_forward_hostio_batches(shape, xs_host, *args, ys_host, ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    for b in range(3):
+        assert torch.equal(ys_host[b], refs[b]), f"batch {b} after the normal call"
+
+
 @pytest.mark.parametrize("T,stall_chunk", [(2048, 0), (2048, 1), (2048, 2), (300, 0)],
                          ids=["first-of-three-chunks", "middle-chunk", "last-chunk", "one-chunk"])
 def test_hostio_reports_a_timeout_in_any_chunk(T, stall_chunk):
