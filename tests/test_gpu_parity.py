@@ -90,6 +90,8 @@ STREAM_ROUTE = {
     "E32k8-d1024": (4097, 1024, 32, 8),
     "E16k4-d2048": (5000, 2048, 16, 4),
     "d1536": (2500, 1536, 8, 2),
+    # rings 4 slots deep refilled: 5-6 tiles of 14 rows per CTA at d = 1024
+    "depth4-reuse-d1024": (12000, 1024, 8, 2),
 }
 
 
@@ -313,8 +315,8 @@ def test_hostio_token_chunks_equal_the_whole_batch(T):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
 
 
-@pytest.mark.parametrize("T,E,k", [(3200, 5, 3), (4097, 32, 8), (3500, 16, 4)],
-                         ids=["E5k3", "E32k8", "E16k4"])
+@pytest.mark.parametrize("T,E,k", [(3200, 5, 3), (4097, 32, 8), (3500, 16, 4), (12000, 8, 2)],
+                         ids=["E5k3", "E32k8", "E16k4", "E8k2-deep-rings"])
 def test_hostio_chunks_route_alike_in_both_router_kernels(T, E, k):
     """The host-I/O pipeline routes its small edge chunks through the cluster
     router (C = 1, the whole batch's split) and its large middle chunk through
