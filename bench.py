@@ -79,13 +79,27 @@ def parse(argv=None):
 
 
 def load_peaks():
+    """The measured copy bandwidth and bf16 GEMM rates of this machine's B200s from
+    MEASURED_PEAKS.json (hbm_gbs, bf16_tflops, bf16_tflops_sustained), each
+    missing or non-numeric entry replaced by the earlier measurement in
+    FALLBACK_PEAKS; the second value says which ("measured", "partly measured",
+    "fallback")."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peaks = dict(FALLBACK_PEAKS)
     try:
         with open(path) as f:
-            p = json.load(f)
-        return p, "measured"
+            found = json.load(f)
     except (OSError, ValueError):
-        return dict(FALLBACK_PEAKS), "fallback"
+        return peaks, "fallback"
+    got = 0
+    for key in FALLBACK_PEAKS:
+        v = found.get(key) if isinstance(found, dict) else None
+        if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+            peaks[key] = float(v)
+            got += 1
+    if got == len(FALLBACK_PEAKS):
+        return peaks, "measured"
+    return peaks, ("partly measured" if got else "fallback")
 
 
 def source_hash():
