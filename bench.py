@@ -45,7 +45,8 @@ SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 KERNEL_SOURCES = ["sparse_mixture_experts_05_b200/csrc/expert_gemm.cu",
                   "sparse_mixture_experts_05_b200/csrc/sm100.cuh",
-                  "sparse_mixture_experts_05_b200/csrc/common.cuh"]
+                  "sparse_mixture_experts_05_b200/csrc/common.cuh",
+                  "sparse_mixture_experts_05_b200/csrc/combine_math.cuh"]
 
 
 def parse(argv=None):

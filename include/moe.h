@@ -178,6 +178,9 @@ int moe_combine(moe_shape s, const float* o, const int32_t* inv, const float* ga
  *   x, Wg, bias (nullable), W1, W3, W2 as above (in);  y [T,d] bf16 (out)
  *   idx_out [T,k] int32, gate_out [T,k] float: copies of the routing, or NULL
  *   ws: >= moe_forward_workspace_bytes(s) bytes of device memory
+ * y has the bits of moe_route -> moe_dispatch -> moe_expert_swiglu -> moe_combine
+ * on the same inputs; at large batches (16 or more rounds of the down
+ * projection's CTA-pair tiles) the combine runs inside that GEMM's epilogue.
  */
 int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, const void* W1,
                 const void* W3, const void* W2, void* y, int32_t* idx_out, float* gate_out,
@@ -200,7 +203,9 @@ int moe_forward_bias(moe_shape s, const void* x, const void* Wg, const float* bi
  * seven caller-created CUDA events (cudaEvent_t handles) on `stream` between its
  * launches: events[0] before the router, [1] after the router, [2] after the
  * dispatch index kernel, [3] after the dispatch scatter, [4] after GEMM1
- * (x W1 | x W3 -> h), [5] after GEMM2 (h W2 -> o), [6] after the combine.
+ * (x W1 | x W3 -> h), [5] after GEMM2 (h W2 -> o), [6] after the combine
+ * (right after [5] when the batch is large enough for the combine to run in
+ * GEMM2's epilogue: at least 16 rounds of its CTA-pair tiles).
  * n_events must be 7.  Measurement hook with no counterpart on the pages.
  */
 int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float* bias,

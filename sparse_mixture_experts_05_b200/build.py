@@ -20,7 +20,7 @@ LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["api.cu", "router.cu", "dispatch.cu", "expert_gemm.cu", "combine.cu", "aux_loss.cu",
            "tma_map.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "expert_gemm.cuh", "router.cuh", "dispatch.cuh",
-           "combine.cuh", "aux_loss.cuh", "tma_map.cuh"]
+           "combine.cuh", "combine_math.cuh", "aux_loss.cuh", "tma_map.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -54,7 +54,7 @@ bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 
 // Workspace of moe_forward, in order; every segment starts on a 256-byte boundary.
 struct FwdLayout {
-    size_t hdr, idx, gate, offsets, perm, inv, x_sorted, h, o, total;
+    size_t hdr, idx, gate, offsets, perm, inv, x_sorted, h, o, cnt, total;
 };
 
 FwdLayout fwd_layout(const moe_shape& s) {
@@ -75,6 +75,8 @@ FwdLayout fwd_layout(const moe_shape& s) {
     L.x_sorted = take(R * s.d * 2);
     L.h = take(R * s.d_ff * 2);
     L.o = take(R * s.d * 4);
+    // counters of the combine fused into the down projection (when it can be)
+    L.cnt = take(combine_fusable(s) ? T * (s.d / 128) * 4 : 0);
     L.total = off;
     return L;
 }
@@ -106,7 +108,8 @@ struct FwdOptions {
 
 // Records events[i] (when given) between the launches: 0 before the router, 1
 // after it, 2 after the dispatch index kernel, 3 after the scatter, 4 after
-// GEMM1, 5 after GEMM2, 6 after the combine.
+// GEMM1, 5 after GEMM2, 6 after the combine (right after 5 when the combine is
+// fused into GEMM2).
 int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias,
                  const void* W1, const void* W3, const void* W2, void* y, int32_t* idx_out,
                  float* gate_out, void* ws, cudaStream_t st, void* const* events,
@@ -133,15 +136,30 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     if (rc) return rc;
     if (!mark(2)) return MOE_ERR_CUDA;
     // the experts' rows: the layer input, or the router's normalised rows u
-    rc = launch_dispatch_scatter(s, opt.norm ? opt.norm->u : x, inv, xs, st);
+    // A routed batch that gives the down projection several rounds of CTA-pair
+    // tiles has the combine fused into that GEMM's epilogue (same bits, one
+    // launch less).
+    const bool fused = combine_fused(s);
+    int* cnt = fused ? at<int>(ws, L.cnt) : nullptr;
+    rc = launch_dispatch_scatter(s, opt.norm ? opt.norm->u : x, inv, xs, st, cnt);
     if (rc) return rc;
     if (!mark(3)) return MOE_ERR_CUDA;
+    FusedCombine fc;
+    fc.perm_tok = perm;
+    fc.inv = inv;
+    fc.gate = gate;
+    fc.residual = opt.residual;
+    fc.y = y;
+    fc.cnt = cnt;
     rc = expert_gemms(s, xs, offsets, W1, W3, W2, h, o, status, opt.timeout_ns, opt.stall_after,
-                      st, events ? events[4] : nullptr, opt.eb.b1, opt.eb.b3, opt.eb.b2);
+                      st, events ? events[4] : nullptr, opt.eb.b1, opt.eb.b3, opt.eb.b2,
+                      fused ? &fc : nullptr);
     if (rc) return rc;
     if (!mark(5)) return MOE_ERR_CUDA;
-    rc = launch_combine(s, o, inv, gate, y, st, opt.residual);
-    if (rc) return rc;
+    if (!fused) {
+        rc = launch_combine(s, o, inv, gate, y, st, opt.residual);
+        if (rc) return rc;
+    }
     return mark(6) ? MOE_OK : MOE_ERR_CUDA;
 }
 

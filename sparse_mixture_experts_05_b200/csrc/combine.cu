@@ -12,6 +12,7 @@
 #include <algorithm>
 
 #include "combine.cuh"
+#include "combine_math.cuh"
 #include "common.cuh"
 
 namespace moe {
@@ -50,35 +51,28 @@ __global__ void __launch_bounds__(256)
                 v[s][1] = __ldg(src + 1);
             }
         }
-        float acc[8];
-        bool first = true;
+        float vv[KMAX][8];
 #pragma unroll
         for (int s = 0; s < KMAX; ++s) {
-            if (s >= k || rows[s] < 0) continue;
-            const float g = gs[s];
-            const float p[8] = {__fmul_rn(g, v[s][0].x), __fmul_rn(g, v[s][0].y),
-                                __fmul_rn(g, v[s][0].z), __fmul_rn(g, v[s][0].w),
-                                __fmul_rn(g, v[s][1].x), __fmul_rn(g, v[s][1].y),
-                                __fmul_rn(g, v[s][1].z), __fmul_rn(g, v[s][1].w)};
+            if (s >= k) break;
+            const float f[8] = {v[s][0].x, v[s][0].y, v[s][0].z, v[s][0].w,
+                                v[s][1].x, v[s][1].y, v[s][1].z, v[s][1].w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = first ? p[j] : __fadd_rn(acc[j], p[j]);
-            first = false;
+            for (int j = 0; j < 8; ++j) vv[s][j] = f[j];
         }
-        if (first) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-        }
-        if (residual) {  // H = U + MoE(.): one more float32 addition before the rounding
+        float res[8], out[8];
+        if (residual) {
             const uint4 r = __ldg(residual + i);
             const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                acc[2 * j] = __fadd_rn(bf16_lo(w[j]), acc[2 * j]);
-                acc[2 * j + 1] = __fadd_rn(bf16_hi(w[j]), acc[2 * j + 1]);
+                res[2 * j] = bf16_lo(w[j]);
+                res[2 * j + 1] = bf16_hi(w[j]);
             }
         }
-        y[i] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                          pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        combine_columns<KMAX, 8>(vv, gs, rows, k, residual != nullptr, res, out);
+        y[i] = make_uint4(pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]),
+                          pack_bf16x2(out[4], out[5]), pack_bf16x2(out[6], out[7]));
     }
 }
 

@@ -184,10 +184,12 @@ __global__ void __launch_bounds__(kIndexThreads, 1)
 
 // x_sorted[inv[t, s]] = x[t] for every slot s of token t; one thread per
 // (token, 16-byte chunk), so x is read once and the k copies are written with
-// coalesced 16-byte stores however few tokens there are.
+// coalesced 16-byte stores however few tokens there are.  With `cnt`, the
+// thread of every 16th chunk (the first of 128 columns) also zeroes that
+// column chunk's counter.
 __global__ void __launch_bounds__(256)
     scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv, int T, int chunks,
-                   int k, uint4* __restrict__ x_sorted) {
+                   int k, uint4* __restrict__ x_sorted, int* __restrict__ cnt) {
     grid_dependency_wait();
     const int64_t total = (int64_t)T * chunks;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -201,6 +203,7 @@ __global__ void __launch_bounds__(256)
             const int dst = __ldg(inv + (int64_t)t * k + s);
             if (dst >= 0) x_sorted[(int64_t)dst * chunks + c] = v;
         }
+        if (cnt && (c & 15) == 0) cnt[(int64_t)t * (chunks >> 4) + (c >> 4)] = 0;
     }
 }
 
@@ -235,7 +238,7 @@ int launch_dispatch_index(const moe_shape& s, const int32_t* idx, int32_t* offse
 }
 
 int launch_dispatch_scatter(const moe_shape& s, const void* x, const int32_t* inv, void* x_sorted,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, int* cnt) {
     using namespace dispatch;
     if (s.T == 0) return MOE_OK;
     const int64_t work = (int64_t)s.T * (s.d / 8);
@@ -243,7 +246,7 @@ int launch_dispatch_scatter(const moe_shape& s, const void* x, const int32_t* in
                                                                  (int64_t)device_sm_count() * 8));
     return launch_pdl(scatter_kernel, dim3(grid), dim3(256), 0, stream,
                       static_cast<const uint4*>(x), inv, s.T, s.d / 8, s.k,
-                      static_cast<uint4*>(x_sorted)) == cudaSuccess
+                      static_cast<uint4*>(x_sorted), cnt) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

@@ -44,6 +44,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "combine_math.cuh"
 #include "expert_gemm.cuh"
 #include "sm100.cuh"
 
@@ -85,6 +86,16 @@ struct Params {
     const float* bias_a;     // GEMM1: b1 [E, n_out]; GEMM2: b2 [E, n_out]; or nullptr
     const float* bias_b;     // GEMM1: b3 [E, n_out]; or nullptr
     int halves_inline;       // pair kernel: half tiles in place (1) or after all full tiles (0)
+    // GEMM2 on CTA pairs with the combine fused (y non-null): besides o, each
+    // token's 128-column chunks of y, finished by whichever of its k row tiles
+    // stores last (see finish_tokens)
+    const int32_t* perm_tok;  // [R] token of each sorted row
+    const int32_t* inv;       // [T, k] sorted row of each (token, slot)
+    const float* gate;        // [T, k]
+    const void* residual;     // [T, n_out] bf16 added before the rounding, or nullptr
+    void* y;                  // [T, n_out] bf16, or nullptr: o only
+    int* cnt;                 // [T, n_out / 128] o stores done per chunk, zero at launch
+    int k;
 };
 
 // Tiles are dealt round-robin to `active` workers (CTAs, or CTA pairs): the
@@ -301,6 +312,136 @@ __device__ __forceinline__ void epilogue_store_f32(uint32_t taddr, bool valid, b
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 dst[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        }
+    }
+}
+
+__device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_ca8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The combine fused into the down projection's epilogue.  A warp has just
+// stored o for its 32 rows (one per lane) and `ncols` columns from x0 (1 or 2
+// chunks of 128).  A (token, chunk) of y needs the o rows of all k of the
+// token's slots, stored by k row tiles in any order.  Once its own stores are
+// complete and visible, each lane counts its chunks done with one atomic add
+// per chunk; a lane whose add is the k-th holds the token's last rows, and the
+// warp then forms those chunks of y together, 4 columns a lane, with the
+// combine kernel's arithmetic (so y has the same bits as with the separate
+// combine).  The rows come from L2 through asynchronous copies into the warp's
+// idle staging buffers (`stage`, kEpiWarpBytes), as many chunks' rows at once
+// as fit, so the loads' latency is paid once per batch of chunks.  Nothing
+// waits on another CTA.  Every slot of a routed token has a row (the router
+// always selects k experts), so k adds finish it.
+template <int KMAX>
+__device__ __noinline__ void finish_tokens(const Params& p, uint8_t* stage, bool valid, bool tma,
+                                           int64_t grow, int x0, int ncols, int lane) {
+    // the warp's TMA stores (issued by lane 0) complete: their rows are in
+    // memory and the staging buffers are free
+    if (lane == 0) {
+        bulk_wait_group<0>();
+        if (tma) fence_proxy_async_global();
+    }
+    __syncwarp();
+    __threadfence();  // this warp's o stores before its counts
+    const int chunks = p.n_out >> 7;
+    const int tok = valid ? __ldg(p.perm_tok + grow) : 0;
+    unsigned m[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        bool mine = false;
+        if (valid && j * 128 < ncols) {
+            const int old = atomicAdd(p.cnt + (int64_t)tok * chunks + (x0 >> 7) + j, 1);
+            mine = old == p.k - 1;
+        }
+        m[j] = __ballot_sync(0xffffffffu, mine);
+    }
+    if ((m[0] | m[1]) == 0u) return;
+    __threadfence();  // the other tiles' counts before their rows
+    // each lane's token's sorted rows and gates, handed to the warp by shuffles
+    int my_rows[KMAX];
+    float my_gs[KMAX];
+    const bool any = ((m[0] | m[1]) >> lane) & 1u;
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+        const bool in = any && s < p.k;
+        my_rows[s] = in ? __ldg(p.inv + (int64_t)tok * p.k + s) : -1;
+        my_gs[s] = in ? __ldg(p.gate + (int64_t)tok * p.k + s) : 0.f;
+    }
+    const float* o = static_cast<const float*>(p.out);
+    const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(p.residual);
+    uint2* y = static_cast<uint2*>(p.y);
+    const int n4 = p.n_out >> 2;
+    // per chunk: k rows of 32 lanes x 16 bytes, then 32 x 8 bytes of residual
+    const int item_bytes = p.k * 512 + (res ? 256 : 0);
+    const int per_batch = kEpiWarpBytes / item_bytes;
+    const uint32_t sbase = smem_u32(stage);
+#pragma unroll 1
+    while ((m[0] | m[1]) != 0u) {  // warp-uniform
+        const unsigned b0 = m[0], b1 = m[1];
+        int n = 0;
+        // issue: the next per_batch (lane, chunk) items' rows
+#pragma unroll 1
+        for (; n < per_batch && (m[0] | m[1]) != 0u; ++n) {
+            const int j = m[0] ? 0 : 1;
+            const int src = __ffs(m[j]) - 1;
+            m[j] &= m[j] - 1;
+            const int col = x0 + j * 128 + lane * 4;  // this lane's 4 columns
+            const uint32_t at = sbase + (uint32_t)(n * item_bytes);
+#pragma unroll
+            for (int s = 0; s < KMAX; ++s) {
+                if (s >= p.k) break;
+                const int row = __shfl_sync(0xffffffffu, my_rows[s], src);
+                if (row >= 0) cp_async_cg16(at + s * 512 + lane * 16, o + (int64_t)row * p.n_out + col);
+            }
+            if (res) {
+                const int t = __shfl_sync(0xffffffffu, tok, src);
+                cp_async_ca8(at + p.k * 512 + lane * 8, res + (int64_t)t * p.n_out + col);
+            }
+        }
+        cp_async_wait_all();
+        // combine: the same items in the same order
+        unsigned q[2] = {b0, b1};
+#pragma unroll 1
+        for (int u = 0; u < n; ++u) {
+            const int j = q[0] ? 0 : 1;
+            const int src = __ffs(q[j]) - 1;
+            q[j] &= q[j] - 1;
+            const int col = x0 + j * 128 + lane * 4;
+            const int t = __shfl_sync(0xffffffffu, tok, src);
+            const uint8_t* at = stage + u * item_bytes;
+            int rows[KMAX];
+            float gs[KMAX];
+            float v[KMAX][4];
+#pragma unroll
+            for (int s = 0; s < KMAX; ++s) {
+                rows[s] = __shfl_sync(0xffffffffu, my_rows[s], src);
+                gs[s] = __shfl_sync(0xffffffffu, my_gs[s], src);
+                if (s < p.k && rows[s] >= 0) {
+                    const float4 f = *reinterpret_cast<const float4*>(at + s * 512 + lane * 16);
+                    v[s][0] = f.x;
+                    v[s][1] = f.y;
+                    v[s][2] = f.z;
+                    v[s][3] = f.w;
+                }
+            }
+            float r[4], out[4];
+            if (res) {
+                const uint2 w = *reinterpret_cast<const uint2*>(at + p.k * 512 + lane * 8);
+                r[0] = bf16_lo(w.x);
+                r[1] = bf16_hi(w.x);
+                r[2] = bf16_lo(w.y);
+                r[3] = bf16_hi(w.y);
+            }
+            combine_columns<KMAX, 4>(v, gs, rows, p.k, res != nullptr, r, out);
+            y[(int64_t)t * n4 + (col >> 2)] =
+                make_uint2(pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]));
         }
     }
 }
@@ -570,6 +711,12 @@ constexpr int kPairBBoxes = 2;                                 // B boxes per CT
 constexpr int kPairStageBytes = kABytes + kPairBBoxes * kBBoxBytes;   // 32 KB
 constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + kEpiBytes + 1024;
 constexpr int kPairMinRows = 512;
+// Rounds of GEMM2 pair tiles from which the combine runs in GEMM2's epilogue.
+// Finishing y there made GEMM2 longer by about as much as the combine kernel
+// took at the Mixtral prefill batch (7 rounds: +27-31 us against 34-36 us, a
+// variant that only counted cost +2 us), and saved 40-95 us a step at the
+// skewed 16384-token batch (28 rounds).
+constexpr int kFuseMinRounds = 16;
 constexpr int kPairMinRounds = 8;
 constexpr int kInlineHalfRounds = 16;
 
@@ -631,7 +778,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmA64,
                             const __grid_constant__ CUtensorMap tmB0,
                             const __grid_constant__ CUtensorMap tmB1,
-                            const __grid_constant__ CUtensorMap tmOut, const Params p) {
+                            const __grid_constant__ CUtensorMap tmOut,
+                            const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -884,6 +1032,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + acc * (uint32_t)sizeof(uint64_t));
+            if (!kSwiGLU && p.y) {  // the accumulator is free again: finish tokens meanwhile
+                const int ncols = pt.half ? boxes * kBoxN : 2 * boxes * kBoxN;
+                const int x0 = pt.ti.n0 + col_half * boxes * kBoxN;
+                if (p.k <= 2)
+                    finish_tokens<2>(p, st.base, valid, tma, grow, x0, ncols, lane);
+                else
+                    finish_tokens<8>(p, st.base, valid, tma, grow, x0, ncols, lane);
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
@@ -1051,10 +1207,25 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& a64, const CUten
 
 }  // namespace gemm
 
+// The fused combine counts whole 128-column chunks per warp: it needs GEMM2 on
+// CTA pairs with 256-column tiles (each warp then stores 1 or 2 whole chunks).
+bool combine_fusable(const moe_shape& s) {
+    return (int64_t)s.T * s.k >= gemm::kPairMinRows && s.d % 256 == 0;
+}
+
+// The combine is fused only when GEMM2 has many rounds of pair tiles
+// (kFuseMinRounds).
+bool combine_fused(const moe_shape& s) {
+    if (!combine_fusable(s)) return false;
+    const int64_t tiles = ((int64_t)s.T * s.k / gemm::kPM) * (s.d / 256);
+    return tiles >= (int64_t)gemm::kFuseMinRounds * std::max(1, device_sm_count() / 2);
+}
+
 int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offsets, const void* W1,
                  const void* W3, const void* W2, void* h, float* o, int* err,
                  uint64_t timeout_ns, int stall_after, cudaStream_t stream,
-                 void* mid_event, const float* b1, const float* b3, const float* b2) {
+                 void* mid_event, const float* b1, const float* b3, const float* b2,
+                 const FusedCombine* fuse) {
     using namespace gemm;
     const int R = s.T * s.k;
     if (R == 0) return MOE_OK;
@@ -1144,6 +1315,15 @@ int expert_gemms(const moe_shape& s, const void* x_sorted, const int32_t* offset
     p2.bias_a = b2;
     p2.bias_b = nullptr;
     p2.halves_inline = inline_halves(p2.n_tile_out, s.d);
+    p2.k = s.k;
+    if (fuse && combine_fusable(s)) {
+        p2.perm_tok = fuse->perm_tok;
+        p2.inv = fuse->inv;
+        p2.gate = fuse->gate;
+        p2.residual = fuse->residual;
+        p2.y = fuse->y;
+        p2.cnt = fuse->cnt;
+    }
     if (!make_weight_map(&m2, W2, (uint64_t)s.E * s.d_ff, (uint64_t)s.d, (uint32_t)p2.n_boxes))
         return MOE_ERR_CUDA;
     const int t2 = mtiles(pairs2 ? kPM : kBM) * (s.d / p2.n_tile_out);

@@ -1,0 +1,113 @@
+"""The combine fused into the down projection's epilogue, bit for bit.
+
+When a routed batch gives the down projection (on CTA pairs, 256-row and
+256-column tiles, d a multiple of 256) at least 16 rounds of pair tiles on the
+device's SMs, that GEMM forms y itself: the last of a token's k row tiles to
+store its o rows adds the token's gate-weighted rows up.  That y must have
+exactly the bits of the separate path (dispatch, experts, combine through
+their own entry points), and of a float32 model of the combine's arithmetic
+written here in numpy: products rounded to float32, summed in slot order, the
+block's residual added last, one rounding to bf16 (nearest even).  The cases
+below have 1184 or more pair tiles (16 rounds of 74 pairs on 148 SMs) unless
+marked otherwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sparse_mixture_experts_05_b200 as moe
+from sparse_mixture_experts_05_b200.inputs import make_inputs
+
+from _parity import to_dev, u16
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # name: (T, d, d_ff, E, k, seed, bias)
+    "k1": (19200, 4096, 256, 8, 1, 31, False),
+    "k2": (9600, 4096, 256, 8, 2, 32, True),
+    "k2-d768": (50600, 768, 256, 8, 2, 33, False),     # 3 column tiles of 256
+    "k2-d2048": (19000, 2048, 256, 8, 2, 34, False),
+    "E5k3": (6400, 4096, 256, 5, 3, 35, False),
+    "E16k4": (4800, 4096, 256, 16, 4, 36, False),
+    "E32k8": (4800, 2048, 256, 32, 8, 37, False),      # the largest E and k (and d for E = 32)
+    "E1k1": (19044, 4096, 256, 1, 1, 38, False),       # 74 full pair tiles and a half tile
+    # not fused: d not a multiple of 256, fewer than 512 rows, under 16 rounds
+    "d384": (1400, 384, 256, 8, 2, 39, False),
+    "small": (200, 256, 256, 8, 2, 40, False),
+    "rounds": (4096, 4096, 256, 8, 2, 41, False),      # the prefill batch's 7 rounds
+}
+
+
+def _round_bf16(a32: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bits, round to nearest even (finite inputs)."""
+    u = a32.astype(np.float32).view(np.uint32).astype(np.uint64)
+    u = u + 0x7FFF + ((u >> 16) & 1)
+    return (u >> 16).astype(np.uint16)
+
+
+def _combine_model(o32, inv, gate, residual_bits=None):
+    acc = None
+    for s in range(inv.shape[1]):
+        p = gate[:, s:s + 1].astype(np.float32) * o32[inv[:, s]]
+        acc = p if acc is None else acc + p
+    if residual_bits is not None:
+        res = (residual_bits.astype(np.uint32) << 16).view(np.float32)
+        acc = res + acc
+    return _round_bf16(acc)
+
+
+def _split_path(shape, x, idx, gate, dev):
+    """dispatch -> experts -> combine, each through its own entry point."""
+    offsets, perm, inv, xs = moe.moe_dispatch(shape, idx, x)
+    _, o, _ = moe.moe_expert_swiglu(shape, xs, offsets, dev["W1"], dev["W3"], dev["W2"])
+    y = moe.moe_combine(shape, o, inv, gate)
+    return y, o, inv
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_combine_equals_the_separate_path(name):
+    T, d, d_ff, E, k, seed, bias = CASES[name]
+    inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    shape = inp["shape"]
+    dev = to_dev(inp)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ws = moe.workspace(moe.moe_forward_workspace_bytes(shape), "cuda")
+    # twice on one workspace: the counters are zeroed again for the second call
+    for _ in range(2):
+        y = moe.moe_forward(shape, dev["x"], dev["Wg"], dev["bias"], dev["W1"], dev["W3"],
+                            dev["W2"], idx_out=idx, gate_out=gate, ws=ws)
+        torch.cuda.synchronize()
+        assert moe.moe_read_device_status(ws) == moe.MOE_OK
+        y_split, o, inv = _split_path(shape, dev["x"], idx, gate, dev)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_split)
+    model = _combine_model(o.cpu().numpy(), inv.cpu().numpy(), gate.cpu().numpy())
+    assert np.array_equal(u16(y), model)
+
+
+@pytest.mark.parametrize("name", ["k2", "E16k4", "d384"])
+def test_fused_combine_adds_the_block_residual(name):
+    """H = U + MoE(u) with u = RMSNorm(U): H against the float32 model on the
+    separate path's rows, routed from the u the block left in its workspace."""
+    T, d, d_ff, E, k, seed, bias = CASES[name]
+    inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    shape = inp["shape"]
+    dev = to_dev(inp)
+    rng = np.random.default_rng(seed)
+    gamma = torch.from_numpy((1 + 0.2 * rng.standard_normal(d)).astype(np.float32))
+    gamma = gamma.to(torch.bfloat16).cuda()
+    ws = moe.workspace(moe.moe_block_workspace_bytes(shape), "cuda")
+    H = moe.moe_block_forward(shape, dev["x"], gamma, dev["Wg"], dev["bias"], dev["W1"],
+                              dev["W3"], dev["W2"], eps=1e-5, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    off = moe.moe_forward_workspace_bytes(shape)
+    u = ws[off:off + T * d * 2].view(torch.bfloat16).view(T, d).clone()
+    idx, gate = moe.moe_route(shape, u, dev["Wg"], dev["bias"])[:2]
+    _, o, inv = _split_path(shape, u, idx, gate, dev)
+    torch.cuda.synchronize()
+    model = _combine_model(o.cpu().numpy(), inv.cpu().numpy(), gate.cpu().numpy(),
+                           residual_bits=u16(inp["x"]))
+    assert np.array_equal(u16(H), model)
