@@ -767,7 +767,7 @@ def run_ours(a):
                                 "ms_per_step": round(e2e_single_ms, 4),
                                 "api": "moe_forward_hostio once per step (three token chunks "
                                        "inside the call), L2 flushed before each"}},
-        "gpu_launches": 6 * a.steps,
+        "gpu_launches": moe.moe_forward_kernel_count(ctx["shape"]) * a.steps,
         "clocks": clocks,
         "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
         "ms_per_step_profiled": round(p_max_ms, 4),

@@ -84,6 +84,14 @@ size_t moe_expert_workspace_bytes(moe_shape s);
  * intermediate of the layer plus the moe_expert_swiglu workspace). */
 size_t moe_forward_workspace_bytes(moe_shape s);
 
+/* Number of kernels one moe_forward (or moe_block_forward) of shape s launches
+ * on the current device: router, dispatch index, dispatch scatter, the two
+ * expert GEMMs, and the combine unless the down projection forms y itself
+ * (16 or more rounds of its CTA-pair tiles on this device's SMs).  0 for
+ * T == 0; a negative status (-MOE_ERR_...) for a shape moe_forward rejects.
+ * Queries the device's SM count; launches nothing. */
+int moe_forward_kernel_count(moe_shape s);
+
 /*
  * moe_route -- router, top-k and softmax over the selected k.
  * Page: section "Прямой проход в формулах" (g = u W_r, S = TopK(g, k), w_i) and

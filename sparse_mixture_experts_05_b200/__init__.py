@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     moe_forward_hostio_batches_stall_test, moe_forward_hostio_batches_workspace_bytes,
     moe_forward_hostio_stall_test,
     moe_forward_hostio_workspace_bytes,
-    moe_forward_profiled, moe_forward_static, moe_forward_workspace_bytes,
+    moe_forward_kernel_count, moe_forward_profiled, moe_forward_static,
+    moe_forward_workspace_bytes,
     moe_read_device_status, moe_route, status_string, workspace,
 )

@@ -27,7 +27,8 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 # Entry points declared in include/moe.h.
 EXPORTS = (
     "moe_status_string", "moe_check_shape", "moe_expert_workspace_bytes",
-    "moe_forward_workspace_bytes", "moe_forward_hostio_workspace_bytes", "moe_route",
+    "moe_forward_workspace_bytes", "moe_forward_kernel_count", "moe_forward_hostio_workspace_bytes",
+    "moe_route",
     "moe_dispatch", "moe_expert_swiglu", "moe_expert_swiglu_bias", "moe_expert_swiglu_stall_test",
     "moe_combine", "moe_forward", "moe_forward_bias", "moe_forward_profiled", "moe_forward_hostio", "moe_forward_hostio_stall_test",
     "moe_forward_hostio_batches_workspace_bytes", "moe_forward_hostio_batches",
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
                    "moe_forward_hostio_batches_workspace_bytes"):
             getattr(L, fn).restype = Z
             getattr(L, fn).argtypes = [S]
+        L.moe_forward_kernel_count.restype = I
+        L.moe_forward_kernel_count.argtypes = [S]
         L.moe_route.restype = I
         L.moe_route.argtypes = [S, P, P, P, P, P, P, P]
         L.moe_dispatch.restype = I
@@ -166,6 +169,15 @@ def moe_expert_workspace_bytes(shape) -> int:
 
 def moe_forward_workspace_bytes(shape) -> int:
     return lib().moe_forward_workspace_bytes(_shape(shape))
+
+
+def moe_forward_kernel_count(shape) -> int:
+    """Kernels one moe_forward of `shape` launches on the current device (5 or 6; 0 for
+    T == 0); MoeError for a shape moe_forward rejects."""
+    n = lib().moe_forward_kernel_count(_shape(shape))
+    if n < 0:
+        _check("moe_forward_kernel_count", -n)
+    return n
 
 
 def moe_forward_hostio_workspace_bytes(shape) -> int:

@@ -412,6 +412,12 @@ size_t moe_forward_workspace_bytes(moe_shape s) {
     return fwd_layout(s).total;
 }
 
+int moe_forward_kernel_count(moe_shape s) {
+    if (const int rc = check_shape(s)) return -rc;
+    if (s.T == 0) return 0;
+    return combine_fused(s) ? 5 : 6;
+}
+
 size_t moe_block_workspace_bytes(moe_shape s) {
     if (check_shape(s)) return 0;
     return fwd_layout(s).total + align_up((size_t)s.T * s.d * 2, 256);

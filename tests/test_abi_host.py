@@ -69,6 +69,21 @@ def test_workspace_sizes():
     assert moe.moe_forward_workspace_bytes((80, 4096, 14336, 8, 2)) > binding.MOE_STATIC_SCRATCH_BYTES
 
 
+def test_forward_kernel_count():
+    """Six kernels, five once the down projection forms y itself (16 or more
+    rounds of its CTA-pair tiles; the host without a GPU assumes the B200's
+    148 SMs, 74 pairs), none for an empty batch, an error for a rejected shape."""
+    assert moe.moe_forward_kernel_count((4096, 4096, 14336, 8, 2)) == 6    # 512 pair tiles
+    assert moe.moe_forward_kernel_count((16, 4096, 14336, 8, 2)) == 6      # single CTAs
+    assert moe.moe_forward_kernel_count((16384, 4096, 14336, 8, 2)) == 5   # 2048 pair tiles
+    assert moe.moe_forward_kernel_count((50600, 384, 256, 8, 2)) == 6      # d not a multiple of 256
+    assert moe.moe_forward_kernel_count((0, 128, 256, 8, 2)) == 0
+    with pytest.raises(moe.MoeError):
+        moe.moe_forward_kernel_count((64, 128, 256, 8, 9))
+    assert binding.lib().moe_forward_kernel_count(binding.MoeShape(64, 100, 256, 8, 2)) == \
+        -moe.MOE_ERR_UNSUPPORTED
+
+
 def _call(fn, *args):
     return getattr(binding.lib(), fn)(*args)
 

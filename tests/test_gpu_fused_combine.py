@@ -111,3 +111,36 @@ def test_fused_combine_adds_the_block_residual(name):
     model = _combine_model(o.cpu().numpy(), inv.cpu().numpy(), gate.cpu().numpy(),
                            residual_bits=u16(inp["x"]))
     assert np.array_equal(u16(H), model)
+
+
+def _our_kernels(fn):
+    """Names of this library's kernels (namespace moe) that `fn` launches, from the
+    profiler's CUDA activity."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events()]
+    if not names:
+        pytest.skip("the profiler recorded no CUDA activity")
+    return [n for n in names if "moe::" in n]
+
+
+@pytest.mark.parametrize("name", ["k2", "rounds", "small"])
+def test_forward_kernel_count_matches_the_launches(name):
+    """moe_forward_kernel_count: 5 kernels where the down projection forms y
+    itself, 6 elsewhere, and no combine kernel among the 5."""
+    T, d, d_ff, E, k, seed, bias = CASES[name]
+    inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    shape = inp["shape"]
+    dev = to_dev(inp)
+    ws = moe.workspace(moe.moe_forward_workspace_bytes(shape), "cuda")
+    run = lambda: moe.moe_forward(shape, dev["x"], dev["Wg"], dev["bias"], dev["W1"],  # noqa: E731
+                                  dev["W3"], dev["W2"], ws=ws)
+    run()
+    kernels = _our_kernels(run)
+    n = moe.moe_forward_kernel_count(shape)
+    assert len(kernels) == n, kernels
+    assert (n == 5) == (name == "k2")
+    assert any("combine_kernel" in s for s in kernels) == (n == 6)
