@@ -144,3 +144,35 @@ def test_forward_kernel_count_matches_the_launches(name):
     assert len(kernels) == n, kernels
     assert (n == 5) == (name == "k2")
     assert any("combine_kernel" in s for s in kernels) == (n == 6)
+
+
+@pytest.mark.parametrize("stall_after", [0, 40], ids=["at-once", "after-some-tiles"])
+def test_fused_combine_timeout_in_a_queue_of_batches(stall_after):
+    """The error path with the combine inside GEMM2: in the middle batch of a
+    queue the expert producers stop (at once, or after 40 stages: GEMM1 stalls in
+    its first tiles, GEMM2 after about ten, some tokens' counters already
+    counted).  The call must report MOE_ERR_DEVICE_TIMEOUT, the other batches'
+    y must be exact, and a normal call on the same workspace afterwards (which
+    zeroes the counters again) must be exact and report MOE_OK."""
+    T, d, d_ff, E, k, seed, bias = CASES["k2"]
+    inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    shape = inp["shape"]
+    assert moe.moe_forward_kernel_count(shape) == 5
+    dev = to_dev(inp)
+    args = (dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    g = torch.Generator().manual_seed(57)
+    xs = [(inp["x"].float() + 0.3 * b * torch.randn(T, d, generator=g)).to(torch.bfloat16)
+          for b in range(3)]
+    refs = [moe.moe_forward(shape, x.cuda(), *args).cpu() for x in xs]
+    xs_host = [x.pin_memory() for x in xs]
+    ys_host = [torch.zeros(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    ws = moe.workspace(moe.moe_forward_hostio_batches_workspace_bytes(shape), "cuda")
+    moe.moe_forward_hostio_batches_stall_test(shape, xs_host, *args, ys_host, ws, stall_batch=1,
+                                              stall_after=stall_after, timeout_ns=2_000_000)
+    assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    for b in (0, 2):
+        assert torch.equal(ys_host[b], refs[b]), f"batch {b}"
+    moe.moe_forward_hostio_batches(shape, xs_host, *args, ys_host, ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    for b in range(3):
+        assert torch.equal(ys_host[b], refs[b]), f"batch {b} after the normal call"
