@@ -264,19 +264,25 @@ int moe_forward_hostio(moe_shape s, const void* x_host, const void* Wg, const fl
  * of T tokens each with the same weights, batch b read from the host buffer
  * x_host[b] and written to the host buffer y_host[b] (pinned memory gives
  * asynchronous copies); the loop of a server that feeds the layer a queue of
- * batches.  Each batch runs the whole layer once on `stream` (the weights are
- * streamed once per batch, not once per token chunk); batch b+1's upload and
- * batch b-1's download run on the library's two copy streams while batch b
- * computes, through two staging slots in ws, so only the first upload and the
- * last download are not overlapped.  y_host[b] equals moe_forward on x_host[b]
- * bit for bit.  Everything is ordered after earlier work on `stream`, and
- * `stream` after the last download.  The status word is cleared once, before
- * the first batch, so an expired wait in any batch stays reported.
+ * batches.  Each batch runs the whole layer once (the weights are streamed once
+ * per batch, not once per token chunk), on `stream`; for small batches
+ * (T*k*d*d_ff < 2^34, e.g. decode-sized ones) odd batches run on a second,
+ * library-owned compute stream with their own part of ws, so two consecutive
+ * batches' short kernels overlap; batch
+ * b+1's upload and batch b-1's download run on the library's two copy streams
+ * while batch b computes, through two staging slots each for x and y in ws, so
+ * only the first upload and the last download are not overlapped.  y_host[b]
+ * equals moe_forward on x_host[b] bit for bit.  Everything is ordered after
+ * earlier work on `stream`, and `stream` after the last download and the
+ * second compute stream's last layer.  The status word (at the start of ws) is
+ * cleared once, before the first batch, and every layer reports into it, so an
+ * expired wait in any batch stays reported.
  *   x_host, y_host: arrays of n_batches host pointers (none null), each buffer
  *       T*d bf16, row-major; a buffer may appear more than once (the caller
  *       owns the data order: y_host[b] is written when batch b's download runs).
- *   ws: >= moe_forward_workspace_bytes(s) + 2 x-staging + 2 y-staging slots of
- *       T*d*2 bytes; moe_forward_hostio_batches_workspace_bytes gives the figure.
+ *   ws: >= moe_forward_workspace_bytes(s) (twice for small batches) + 2
+ *       x-staging + 2 y-staging slots of T*d*2 bytes;
+ *       moe_forward_hostio_batches_workspace_bytes gives the figure.
  * Errors: MOE_ERR_INVALID_ARG for n_batches < 1 or a null array or entry,
  * MOE_ERR_WORKSPACE for a short ws; T == 0 enqueues nothing.
  */

@@ -104,6 +104,7 @@ struct FwdOptions {
     int stall_after = -1;            // test hook: expert producer stops after this many stages
     uint64_t timeout_ns = kDefaultWaitTimeoutNs;  // bound on every device wait
     const RouterNorm* norm = nullptr;  // block edge: x is U, the router forms u = RMSNorm_2(U)
+    int* status = nullptr;           // status word (nullptr: the workspace header's)
 };
 
 // Records events[i] (when given) between the launches: 0 before the router, 1
@@ -126,7 +127,7 @@ int forward_impl(const moe_shape& s, const void* x, const void* Wg, const float*
     void* xs = at<void>(ws, L.x_sorted);
     void* h = at<void>(ws, L.h);
     float* o = at<float>(ws, L.o);
-    int* status = at<int>(ws, L.hdr);
+    int* status = opt.status ? opt.status : at<int>(ws, L.hdr);
     if (!mark(0)) return MOE_ERR_CUDA;
     int rc = launch_router(s, x, Wg, bias, idx, gate, nullptr, st, opt.router_cluster, opt.norm,
                            status, opt.clear_status);
@@ -212,10 +213,12 @@ int hostio_chunks(int T, int (&sizes)[kMaxHostioChunks]) {
 // of the process.  The mutex serialises the enqueueing of one call's pipeline.
 struct CopyStreams {
     cudaStream_t up = nullptr, down = nullptr;
+    // moe_forward_hostio_batches: the second compute stream (odd batches)
+    cudaStream_t comp = nullptr;
     cudaEvent_t ev[2 + 2 * kMaxHostioChunks] = {};
     // moe_forward_hostio_batches: start, x landed in slot 0/1, slot 0/1's layer
-    // done, slot 0/1's y left, end
-    cudaEvent_t evb[8] = {};
+    // done, slot 0/1's y left, copies' end, second compute stream's end
+    cudaEvent_t evb[9] = {};
     std::mutex mu;
 };
 
@@ -228,7 +231,8 @@ CopyStreams* copy_streams() {
     if (!per_device[dev]) {
         CopyStreams* cs = new CopyStreams();
         bool ok = cudaStreamCreateWithFlags(&cs->up, cudaStreamNonBlocking) == cudaSuccess &&
-                  cudaStreamCreateWithFlags(&cs->down, cudaStreamNonBlocking) == cudaSuccess;
+                  cudaStreamCreateWithFlags(&cs->down, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&cs->comp, cudaStreamNonBlocking) == cudaSuccess;
         for (auto& e : cs->ev)
             ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
         for (auto& e : cs->evb)
@@ -326,6 +330,17 @@ int hostio_impl(const moe_shape& s, const void* x_host, const void* Wg, const fl
 // and for batch b-2's y to have left the slot, and its download runs while
 // batch b+1 computes.  Each batch is one whole-batch forward, so the weights
 // are streamed once per batch and y_host[b] equals moe_forward on x_host[b].
+// Whether moe_forward_hostio_batches runs alternate batches on two compute
+// streams: only for batches whose expert GEMMs are small (R d d_ff < 2^34, e.g.
+// the decode batch or the quarter-width one).  Measured on a queue of 20
+// batches, two streams against one: decode 0.421 vs 0.443 ms a batch, quarter
+// width 0.081 vs 0.089, but the Mixtral prefill batch 2.72 vs 2.36 ms -- its
+// persistent GEMM grids, dealt their tiles up front, lose SMs to the other
+// stream's kernels and wait for them.
+bool queue_two_streams(const moe_shape& s) {
+    return (int64_t)s.T * s.k * s.d * (int64_t)s.d_ff < (int64_t(1) << 34);
+}
+
 int hostio_batches_impl(const moe_shape& s, int nb, const void* const* x_host, const void* Wg,
                         const float* bias, const void* W1, const void* W3, const void* W2,
                         void* const* y_host, void* ws, size_t ws_bytes, cudaStream_t st,
@@ -342,16 +357,28 @@ int hostio_batches_impl(const moe_shape& s, int nb, const void* const* x_host, c
     if (ws_bytes < moe_forward_hostio_batches_workspace_bytes(s)) return MOE_ERR_WORKSPACE;
     const size_t io_bytes = (size_t)s.T * s.d * 2;
     const size_t slot = align_up(io_bytes, 256);
-    char* base = static_cast<char*>(ws) + moe_forward_workspace_bytes(s);
+    const size_t fwd = moe_forward_workspace_bytes(s);
+    const bool two = queue_two_streams(s);
+    char* base = static_cast<char*>(ws) + (two ? 2 : 1) * fwd;
+    int* status = at<int>(ws, fwd_layout(s).hdr);  // every layer reports here
     CopyStreams* cs = copy_streams();
     if (!cs) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(cs->mu);
-    cudaEvent_t* ev = cs->evb;  // [0] start, [1+i] x in slot i, [3+i] slot i read, [5+i] y out, [7] end
-    bool ok = cudaEventRecord(ev[0], st) == cudaSuccess &&
+    // Small batches: even batches run on the caller's stream with workspace part
+    // 0, odd ones on a second compute stream with part 1, so one batch's short
+    // kernels overlap the other's.  Large ones all run on the caller's stream.
+    cudaStream_t comp[2] = {st, two ? cs->comp : st};
+    // [0] start, [1+i] x in slot i, [3+i] slot i's layer done, [5+i] y out of
+    // slot i, [7] copies' end, [8] second compute stream's end
+    cudaEvent_t* ev = cs->evb;
+    bool ok = cudaMemsetAsync(status, 0, sizeof(int), st) == cudaSuccess &&
+              cudaEventRecord(ev[0], st) == cudaSuccess &&
               cudaStreamWaitEvent(cs->up, ev[0], 0) == cudaSuccess &&
-              cudaStreamWaitEvent(cs->down, ev[0], 0) == cudaSuccess;
+              cudaStreamWaitEvent(cs->down, ev[0], 0) == cudaSuccess &&
+              cudaStreamWaitEvent(cs->comp, ev[0], 0) == cudaSuccess;
     for (int b = 0; ok && b < nb; ++b) {
         const int i = b & 1;
+        cudaStream_t cst = comp[i];
         char* x_dev = base + (size_t)i * slot;
         char* y_dev = base + (size_t)(2 + i) * slot;
         if (b >= 2) ok = cudaStreamWaitEvent(cs->up, ev[3 + i], 0) == cudaSuccess;
@@ -359,25 +386,29 @@ int hostio_batches_impl(const moe_shape& s, int nb, const void* const* x_host, c
              cudaMemcpyAsync(x_dev, x_host[b], io_bytes, cudaMemcpyHostToDevice, cs->up) ==
                  cudaSuccess &&
              cudaEventRecord(ev[1 + i], cs->up) == cudaSuccess &&
-             cudaStreamWaitEvent(st, ev[1 + i], 0) == cudaSuccess;
-        if (ok && b >= 2) ok = cudaStreamWaitEvent(st, ev[5 + i], 0) == cudaSuccess;
+             cudaStreamWaitEvent(cst, ev[1 + i], 0) == cudaSuccess;
+        if (ok && b >= 2) ok = cudaStreamWaitEvent(cst, ev[5 + i], 0) == cudaSuccess;
         FwdOptions opt;
-        opt.clear_status = b == 0;  // an expired wait in any batch stays reported
+        opt.clear_status = false;  // cleared once above: an expired wait in any batch stays
+        opt.status = status;
         if (b == stall_batch) {
             opt.stall_after = stall_after;
             opt.timeout_ns = timeout_ns;
         }
         ok = ok &&
-             forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr, ws, st,
-                          nullptr, opt) == MOE_OK &&
-             cudaEventRecord(ev[3 + i], st) == cudaSuccess &&
+             forward_impl(s, x_dev, Wg, bias, W1, W3, W2, y_dev, nullptr, nullptr,
+                          static_cast<char*>(ws) + (two ? (size_t)i * fwd : 0), cst, nullptr,
+                          opt) == MOE_OK &&
+             cudaEventRecord(ev[3 + i], cst) == cudaSuccess &&
              cudaStreamWaitEvent(cs->down, ev[3 + i], 0) == cudaSuccess &&
              cudaMemcpyAsync(y_host[b], y_dev, io_bytes, cudaMemcpyDeviceToHost, cs->down) ==
                  cudaSuccess &&
              cudaEventRecord(ev[5 + i], cs->down) == cudaSuccess;
     }
     ok = ok && cudaEventRecord(ev[7], cs->down) == cudaSuccess &&
-         cudaStreamWaitEvent(st, ev[7], 0) == cudaSuccess;
+         cudaEventRecord(ev[8], cs->comp) == cudaSuccess &&
+         cudaStreamWaitEvent(st, ev[7], 0) == cudaSuccess &&
+         cudaStreamWaitEvent(st, ev[8], 0) == cudaSuccess;
     return ok ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -432,7 +463,8 @@ size_t moe_forward_hostio_workspace_bytes(moe_shape s) {
 size_t moe_forward_hostio_batches_workspace_bytes(moe_shape s) {
     if (check_shape(s)) return 0;
     const size_t io = align_up((size_t)s.T * s.d * 2, 256);
-    return fwd_layout(s).total + 4 * io;
+    // a forward workspace per compute stream
+    return (queue_two_streams(s) ? 2 : 1) * fwd_layout(s).total + 4 * io;
 }
 
 int moe_route(moe_shape s, const void* x, const void* Wg, const float* bias, int32_t* idx,

@@ -220,7 +220,11 @@ def test_hostio_batches_rejects_bad_arguments_on_host():
     assert _call(fn, S, 2, arr, good, None, good, good, good, holey, good, big, None) == \
         moe.MOE_ERR_INVALID_ARG                                         # a null y entry
     need = moe.moe_forward_hostio_batches_workspace_bytes((64, 128, 256, 8, 2))
-    assert need == moe.moe_forward_workspace_bytes((64, 128, 256, 8, 2)) + 4 * 64 * 128 * 2
+    # small batches: a forward workspace for each of two compute streams
+    assert need == 2 * moe.moe_forward_workspace_bytes((64, 128, 256, 8, 2)) + 4 * 64 * 128 * 2
+    large = (4096, 4096, 14336, 8, 2)  # one compute stream
+    assert moe.moe_forward_hostio_batches_workspace_bytes(large) == \
+        moe.moe_forward_workspace_bytes(large) + 4 * 4096 * 4096 * 2
     assert _call(fn, S, 2, arr, good, None, good, good, good, arr, good,
                  ctypes.c_size_t(need - 1), None) == moe.MOE_ERR_WORKSPACE
     # T = 0 enqueues nothing
