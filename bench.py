@@ -127,19 +127,45 @@ def committed_traffic(workload):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs: through
+    NVML every 2 ms from a thread (a timed region of ten prefill steps lasts about
+    22 ms), else through nvidia-smi every 200 ms.  Reads only; changes nothing."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
 
     def __init__(self, gpu_index: int):
         self.gpu_index = gpu_index
         self.proc = None
         self.lines = []
         self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.samples = []
+        self.done = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            prop = torch.cuda.get_device_properties(self.gpu_index)
+            bus = "%08x:%02x:%02x.0" % (prop.pci_domain_id, prop.pci_bus_id, prop.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index)
 
     def start(self):
+        try:
+            self.nvml, self.handle = self._nvml_handle()
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -151,11 +177,46 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _nvml_loop(self):
+        n = self.nvml
+        while True:
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                why = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((float(sm), int(why)))
+            except Exception:
+                pass
+            if self.done.wait(self.PERIOD_S):
+                return
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    @staticmethod
+    def reasons_of(bits: int):
+        """Names of the throttle reasons in an NVML clock-event bit mask (the ones the
+        measurement rules look at)."""
+        named = [(0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+                 (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown")]
+        return [name for bit, name in named if bits & bit]
+
     def stop(self):
+        if self.nvml is not None:
+            self.done.set()
+            if self.thread:
+                self.thread.join(timeout=2)
+            try:
+                smax = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+            except Exception:
+                smax = None
+            sm = [c for c, _ in self.samples]
+            reasons = set()
+            for _, bits in self.samples:
+                reasons.update(self.reasons_of(bits))
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                    "reasons": sorted(reasons), "samples": len(sm),
+                    "sampler": f"NVML every {self.PERIOD_S * 1000:.0f} ms during the timed region"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -181,7 +242,8 @@ class ClockSampler:
                 if val.lower().startswith("active"):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "sampler": "nvidia-smi every 200 ms"}
 
 
 # ---------------------------------------------------------------- distributed
@@ -338,7 +400,7 @@ def timed_loop(ctx, steps, pg, device, clock, profiled):
 def extras_loop(ctx, steps, device, local):
     """The widened entry points on the same batch, interleaved step by step with
     the plain layer so that all see the same clocks and power state (L2 flushed
-    before every call, nvidia-smi sampled throughout): the block with its edges,
+    before every call, clocks sampled throughout): the block with its edges,
     the layer with expert biases, and the load-balancing term on the router's
     logits.  The order of the five calls rotates by one every step, so each
     call runs in each place equally often over whole rotations (at least 30

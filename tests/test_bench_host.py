@@ -45,3 +45,20 @@ def test_timing_contract_arguments():
     assert bench.parse([]).warmup >= 3
     with pytest.raises(SystemExit):
         bench.parse(["--warmup", "2"])
+
+
+def test_clock_reasons_from_nvml_bits():
+    assert bench.ClockSampler.reasons_of(0) == []
+    assert bench.ClockSampler.reasons_of(0x4) == ["sw_power_cap"]
+    assert bench.ClockSampler.reasons_of(0x4 | 0x8 | 0x20 | 0x40 | 0x80) == [
+        "sw_power_cap", "hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown",
+        "hw_power_brake_slowdown"]
+    assert bench.ClockSampler.reasons_of(0x1 | 0x2) == []   # idle, application clocks
+
+
+def test_clock_sampler_without_a_gpu_reports_no_clock():
+    c = bench.ClockSampler(0)
+    c.start()
+    out = c.stop()
+    assert out["sm_mhz"] is None or out["sm_mhz"] > 0
+    assert "reasons" in out
