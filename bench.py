@@ -525,10 +525,20 @@ def graph_step_ms(ctx, steps):
     return statistics.median(ms), statistics.mean(ms)
 
 
+SETTLE_S = 1.0
+
+
 def secondary_workload(name, steps, warmup, device, rank, local, pg, peaks):
     """A second workload timed like the main one (plain pass with clocks, then the
-    profiled pass for the kernel split) and summarised as an object of the line."""
+    profiled pass for the kernel split) and summarised as an object of the line.
+    It starts after SETTLE_S seconds with the GPU idle, so that it runs in its own
+    power state rather than in the tail of the power limiter's response to the
+    workload before it (the decode batch, which streams weights, measured 0.49-0.50
+    ms at 1387 MHz right after the prefill queue and 0.44 ms at full clock)."""
     w_steps = steps
+    import torch
+    torch.cuda.synchronize()
+    time.sleep(SETTLE_S)
     ctx = time_workload(name, w_steps, warmup, device, rank)
     ms, _, _, clocks = timed_loop(ctx, w_steps, pg, device, ClockSampler(local), profiled=False)
     mean = reduce_max(pg, statistics.mean(ms), device)
@@ -545,7 +555,7 @@ def secondary_workload(name, steps, warmup, device, rank, local, pg, peaks):
            "ms_per_step_max": round(max(ms), 4),
            "kernel_ms": {k_: round(v, 4) for k_, v in parts.items()},
            "ms_per_step_profiled": round(pmean, 4), "expert_rows": ctx["counts"],
-           "clocks": clocks}
+           "clocks": clocks, "settle_s": SETTLE_S}
     if name in ("decode", "quarter", "tiny"):
         g_med, g_mean = graph_step_ms(ctx, w_steps)
         g_med = reduce_max(pg, g_med, device)
