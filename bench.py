@@ -147,16 +147,29 @@ class ClockSampler:
         self.samples = []
         self.done = threading.Event()
 
+    _handles = {}  # gpu index -> (pynvml, handle), looked up once per process
+
+    @classmethod
+    def prepare(cls, gpu_index: int):
+        try:
+            cls(gpu_index)._nvml_handle()
+        except Exception:
+            pass
+
     def _nvml_handle(self):
+        if self.gpu_index in ClockSampler._handles:
+            return ClockSampler._handles[self.gpu_index]
         import pynvml
         pynvml.nvmlInit()
         try:
             import torch
             prop = torch.cuda.get_device_properties(self.gpu_index)
             bus = "%08x:%02x:%02x.0" % (prop.pci_domain_id, prop.pci_bus_id, prop.pci_device_id)
-            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            got = (pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus))
         except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index)
+            got = (pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index))
+        ClockSampler._handles[self.gpu_index] = got
+        return got
 
     def start(self):
         try:
@@ -775,6 +788,7 @@ def run_ours(a):
     peaks, peak_kind = load_peaks()
     moe.binding.lib()
 
+    ClockSampler.prepare(local)  # NVML set up before, not inside, the timed region
     ctx = time_workload(a.workload, a.steps, a.warmup, device, rank, a.tokens, a.experts)
     clock = ClockSampler(local)
     step_ms, _, bracket_ms, clocks = timed_loop(ctx, a.steps, pg, device, clock, profiled=False)
