@@ -176,3 +176,50 @@ def test_fused_combine_timeout_in_a_queue_of_batches(stall_after):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
     for b in range(3):
         assert torch.equal(ys_host[b], refs[b]), f"batch {b} after the normal call"
+
+
+def test_fused_combine_with_expert_biases():
+    """The layer with expert Linear biases (b2 added to o in GEMM2's epilogue
+    before the fused combine reads it): y equals the separate path with the
+    same biases, and the float32 model, bit for bit."""
+    from sparse_mixture_experts_05_b200.inputs import expert_biases
+    T, d, d_ff, E, k, seed, bias = CASES["k2"]
+    inp = make_inputs(T, d, d_ff, E, k, seed, bias=bias)
+    shape = inp["shape"]
+    assert moe.moe_forward_kernel_count(shape) == 5
+    dev = to_dev(inp)
+    eb = tuple(b.cuda() for b in expert_biases(E, d, d_ff, seed=77))
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    y = moe.moe_forward_bias(shape, dev["x"], dev["Wg"], dev["bias"], dev["W1"], dev["W3"],
+                             dev["W2"], eb, idx_out=idx, gate_out=gate)
+    offsets, perm, inv, xs = moe.moe_dispatch(shape, idx, dev["x"])
+    _, o, _ = moe.moe_expert_swiglu_bias(shape, xs, offsets, dev["W1"], dev["W3"], dev["W2"], eb)
+    y_split = moe.moe_combine(shape, o, inv, gate)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_split)
+    model = _combine_model(o.cpu().numpy(), inv.cpu().numpy(), gate.cpu().numpy())
+    assert np.array_equal(u16(y), model)
+
+
+def test_fused_combine_in_token_chunks_equals_the_whole_batch():
+    """moe_forward_hostio cuts a batch of 20000 tokens into chunks of 2496, 15008
+    and 2496 tokens: the middle chunk forms y inside GEMM2, the edge chunks (304
+    pair tiles each) run the combine kernel, and the whole batch (2496 tiles) is
+    fused too; y must be the same bits either way."""
+    T, d, d_ff, E, k = 20000, 4096, 256, 8, 2
+    inp = make_inputs(T, d, d_ff, E, k, 42, bias=True)
+    shape = inp["shape"]
+    assert moe.moe_forward_kernel_count(shape) == 5
+    assert moe.moe_forward_kernel_count((15008, d, d_ff, E, k)) == 5
+    assert moe.moe_forward_kernel_count((2496, d, d_ff, E, k)) == 6
+    dev = to_dev(inp)
+    y = moe.moe_forward(shape, dev["x"], dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
+    x_host = inp["x"].clone().pin_memory()
+    y_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    ws = moe.workspace(moe.moe_forward_hostio_workspace_bytes(shape), "cuda")
+    moe.moe_forward_hostio(shape, x_host, dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"],
+                           y_host, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    assert torch.equal(y.cpu(), y_host)
