@@ -87,7 +87,7 @@ size_t moe_forward_workspace_bytes(moe_shape s);
 /* Number of kernels one moe_forward (or moe_block_forward) of shape s launches
  * on the current device: router, dispatch index, dispatch scatter, the two
  * expert GEMMs, and the combine unless the down projection forms y itself
- * (16 or more rounds of its CTA-pair tiles on this device's SMs).  0 for
+ * (4 or more rounds of its CTA-pair tiles on this device's SMs).  0 for
  * T == 0; a negative status (-MOE_ERR_...) for a shape moe_forward rejects.
  * Queries the device's SM count; launches nothing. */
 int moe_forward_kernel_count(moe_shape s);
@@ -187,7 +187,7 @@ int moe_combine(moe_shape s, const float* o, const int32_t* inv, const float* ga
  *   idx_out [T,k] int32, gate_out [T,k] float: copies of the routing, or NULL
  *   ws: >= moe_forward_workspace_bytes(s) bytes of device memory
  * y has the bits of moe_route -> moe_dispatch -> moe_expert_swiglu -> moe_combine
- * on the same inputs; at large batches (16 or more rounds of the down
+ * on the same inputs; at large batches (4 or more rounds of the down
  * projection's CTA-pair tiles) the combine runs inside that GEMM's epilogue.
  */
 int moe_forward(moe_shape s, const void* x, const void* Wg, const float* bias, const void* W1,
@@ -213,7 +213,7 @@ int moe_forward_bias(moe_shape s, const void* x, const void* Wg, const float* bi
  * dispatch index kernel, [3] after the dispatch scatter, [4] after GEMM1
  * (x W1 | x W3 -> h), [5] after GEMM2 (h W2 -> o), [6] after the combine
  * (right after [5] when the batch is large enough for the combine to run in
- * GEMM2's epilogue: at least 16 rounds of its CTA-pair tiles).
+ * GEMM2's epilogue: at least 4 rounds of its CTA-pair tiles).
  * n_events must be 7.  Measurement hook with no counterpart on the pages.
  */
 int moe_forward_profiled(moe_shape s, const void* x, const void* Wg, const float* bias,

@@ -332,16 +332,19 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // token's slots, stored by k row tiles in any order.  Once its own stores are
 // complete and visible, each lane counts its chunks done with one atomic add
 // per chunk; a lane whose add is the k-th holds the token's last rows, and the
-// warp then forms those chunks of y together, 4 columns a lane, with the
-// combine kernel's arithmetic (so y has the same bits as with the separate
-// combine).  The rows come from L2 through asynchronous copies into the warp's
-// idle staging buffers (`stage`, kEpiWarpBytes), as many chunks' rows at once
-// as fit, so the loads' latency is paid once per batch of chunks.  Nothing
-// waits on another CTA.  Every slot of a routed token has a row (the router
-// always selects k experts), so k adds finish it.
-template <int KMAX>
+// warp then forms those chunks of y with the combine kernel's arithmetic (so y
+// has the same bits as with the separate combine).  The warp works on 32 / LPI
+// chunks at a time, LPI lanes each (128 / LPI columns a lane), so that the
+// chunks' latency chains overlap; their k rows come from L2 through
+// asynchronous copies into the warp's idle staging buffers (`stage`,
+// kEpiWarpBytes), as many chunks at once as fit, then each lane combines the
+// columns it fetched.  Nothing waits on another CTA.  Every slot of a routed
+// token has a row (the router always selects k experts), so k adds finish it.
+template <int KMAX, int LPI>
 __device__ __noinline__ void finish_tokens(const Params& p, uint8_t* stage, bool valid, bool tma,
                                            int64_t grow, int x0, int ncols, int lane) {
+    constexpr int CPL = 128 / LPI;   // columns per lane
+    constexpr int IPS = 32 / LPI;    // chunks per warp step
     // the warp's TMA stores (issued by lane 0) complete: their rows are in
     // memory and the staging buffers are free
     if (lane == 0) {
@@ -352,96 +355,133 @@ __device__ __noinline__ void finish_tokens(const Params& p, uint8_t* stage, bool
     __threadfence();  // this warp's o stores before its counts
     const int chunks = p.n_out >> 7;
     const int tok = valid ? __ldg(p.perm_tok + grow) : 0;
-    unsigned m[2];
+    int old[2] = {-1, -1};
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        bool mine = false;
-        if (valid && j * 128 < ncols) {
-            const int old = atomicAdd(p.cnt + (int64_t)tok * chunks + (x0 >> 7) + j, 1);
-            mine = old == p.k - 1;
-        }
-        m[j] = __ballot_sync(0xffffffffu, mine);
-    }
-    if ((m[0] | m[1]) == 0u) return;
+    for (int j = 0; j < 2; ++j)
+        if (valid && j * 128 < ncols)
+            old[j] = atomicAdd(p.cnt + (int64_t)tok * chunks + (x0 >> 7) + j, 1);
+    const unsigned m0 = __ballot_sync(0xffffffffu, old[0] == p.k - 1);
+    const unsigned m1 = __ballot_sync(0xffffffffu, old[1] == p.k - 1);
+    if ((m0 | m1) == 0u) return;
     __threadfence();  // the other tiles' counts before their rows
-    // each lane's token's sorted rows and gates, handed to the warp by shuffles
+    // each lane's token's sorted rows and gates, handed out by shuffles
     int my_rows[KMAX];
     float my_gs[KMAX];
-    const bool any = ((m[0] | m[1]) >> lane) & 1u;
+    const bool any = ((m0 | m1) >> lane) & 1u;
 #pragma unroll
     for (int s = 0; s < KMAX; ++s) {
         const bool in = any && s < p.k;
         my_rows[s] = in ? __ldg(p.inv + (int64_t)tok * p.k + s) : -1;
         my_gs[s] = in ? __ldg(p.gate + (int64_t)tok * p.k + s) : 0.f;
     }
+    // the chunk list (lane | chunk << 5), chunk 0's in lane order first, in the
+    // last 256 bytes of the staging buffers
+    constexpr int kListBytes = 256;
+    int* list = reinterpret_cast<int*>(stage + kEpiWarpBytes - kListBytes);
+    const unsigned lt = (1u << lane) - 1u;
+    const int n0 = __popc(m0);
+    const int nitems = n0 + __popc(m1);
+    if ((m0 >> lane) & 1u) list[__popc(m0 & lt)] = lane;
+    if ((m1 >> lane) & 1u) list[n0 + __popc(m1 & lt)] = lane | 32;
+    __syncwarp();
     const float* o = static_cast<const float*>(p.out);
     const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(p.residual);
-    uint2* y = static_cast<uint2*>(p.y);
-    const int n4 = p.n_out >> 2;
-    // per chunk: k rows of 32 lanes x 16 bytes, then 32 x 8 bytes of residual
+    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.y);
+    // per chunk: k rows of 128 float32, then 128 bf16 of residual
     const int item_bytes = p.k * 512 + (res ? 256 : 0);
-    const int per_batch = kEpiWarpBytes / item_bytes;
+    const int per_batch = (kEpiWarpBytes - kListBytes) / item_bytes;
     const uint32_t sbase = smem_u32(stage);
+    const int g = lane / LPI;          // this lane's chunk within a step
+    const int qc = (lane % LPI) * CPL;  // and its first column within the chunk
 #pragma unroll 1
-    while ((m[0] | m[1]) != 0u) {  // warp-uniform
-        const unsigned b0 = m[0], b1 = m[1];
-        int n = 0;
-        // issue: the next per_batch (lane, chunk) items' rows
+    for (int base = 0; base < nitems; base += per_batch) {
+        const int nb = min(per_batch, nitems - base);
+        // issue: the batch's chunks' rows (and residual), IPS chunks a step
 #pragma unroll 1
-        for (; n < per_batch && (m[0] | m[1]) != 0u; ++n) {
-            const int j = m[0] ? 0 : 1;
-            const int src = __ffs(m[j]) - 1;
-            m[j] &= m[j] - 1;
-            const int col = x0 + j * 128 + lane * 4;  // this lane's 4 columns
-            const uint32_t at = sbase + (uint32_t)(n * item_bytes);
+        for (int u0 = 0; u0 < nb; u0 += IPS) {
+            const int u = u0 + g;
+            const int e = u < nb ? list[base + u] : 0;
+            const int src = e & 31;
+            const int col = x0 + (e >> 5) * 128 + qc;
+            const uint32_t at = sbase + (uint32_t)(u * item_bytes);
 #pragma unroll
             for (int s = 0; s < KMAX; ++s) {
                 if (s >= p.k) break;
                 const int row = __shfl_sync(0xffffffffu, my_rows[s], src);
-                if (row >= 0) cp_async_cg16(at + s * 512 + lane * 16, o + (int64_t)row * p.n_out + col);
+                if (u < nb && row >= 0) {
+                    const float* from = o + (int64_t)row * p.n_out + col;
+#pragma unroll
+                    for (int c = 0; c < CPL / 4; ++c)
+                        cp_async_cg16(at + s * 512 + qc * 4 + c * 16, from + c * 4);
+                }
             }
             if (res) {
                 const int t = __shfl_sync(0xffffffffu, tok, src);
-                cp_async_ca8(at + p.k * 512 + lane * 8, res + (int64_t)t * p.n_out + col);
+                if (u < nb) {
+                    const __nv_bfloat16* from = res + (int64_t)t * p.n_out + col;
+                    const uint32_t rat = at + p.k * 512 + qc * 2;
+                    if constexpr (CPL >= 8) {
+#pragma unroll
+                        for (int c = 0; c < CPL / 8; ++c) cp_async_cg16(rat + c * 16, from + c * 8);
+                    } else {
+                        cp_async_ca8(rat, from);
+                    }
+                }
             }
         }
-        cp_async_wait_all();
-        // combine: the same items in the same order
-        unsigned q[2] = {b0, b1};
+        cp_async_wait_all();  // each lane reads back only what it fetched
+        // combine: the same chunks, the same lanes
 #pragma unroll 1
-        for (int u = 0; u < n; ++u) {
-            const int j = q[0] ? 0 : 1;
-            const int src = __ffs(q[j]) - 1;
-            q[j] &= q[j] - 1;
-            const int col = x0 + j * 128 + lane * 4;
+        for (int u0 = 0; u0 < nb; u0 += IPS) {
+            const int u = u0 + g;
+            const int e = u < nb ? list[base + u] : 0;
+            const int src = e & 31;
+            const int col = x0 + (e >> 5) * 128 + qc;
             const int t = __shfl_sync(0xffffffffu, tok, src);
             const uint8_t* at = stage + u * item_bytes;
             int rows[KMAX];
             float gs[KMAX];
-            float v[KMAX][4];
+            float v[KMAX][CPL];
 #pragma unroll
             for (int s = 0; s < KMAX; ++s) {
                 rows[s] = __shfl_sync(0xffffffffu, my_rows[s], src);
                 gs[s] = __shfl_sync(0xffffffffu, my_gs[s], src);
-                if (s < p.k && rows[s] >= 0) {
-                    const float4 f = *reinterpret_cast<const float4*>(at + s * 512 + lane * 16);
-                    v[s][0] = f.x;
-                    v[s][1] = f.y;
-                    v[s][2] = f.z;
-                    v[s][3] = f.w;
+                if (u < nb && s < p.k && rows[s] >= 0) {
+#pragma unroll
+                    for (int c = 0; c < CPL / 4; ++c) {
+                        const float4 f =
+                            *reinterpret_cast<const float4*>(at + s * 512 + qc * 4 + c * 16);
+                        v[s][4 * c] = f.x;
+                        v[s][4 * c + 1] = f.y;
+                        v[s][4 * c + 2] = f.z;
+                        v[s][4 * c + 3] = f.w;
+                    }
                 }
             }
-            float r[4], out[4];
+            if (u >= nb) continue;
+            float r[CPL], out[CPL];
             if (res) {
-                const uint2 w = *reinterpret_cast<const uint2*>(at + p.k * 512 + lane * 8);
-                r[0] = bf16_lo(w.x);
-                r[1] = bf16_hi(w.x);
-                r[2] = bf16_lo(w.y);
-                r[3] = bf16_hi(w.y);
+#pragma unroll
+                for (int c = 0; c < CPL / 2; ++c) {
+                    const uint32_t w =
+                        *reinterpret_cast<const uint32_t*>(at + p.k * 512 + qc * 2 + c * 4);
+                    r[2 * c] = bf16_lo(w);
+                    r[2 * c + 1] = bf16_hi(w);
+                }
             }
-            combine_columns<KMAX, 4>(v, gs, rows, p.k, res != nullptr, r, out);
-            y[(int64_t)t * n4 + (col >> 2)] =
-                make_uint2(pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]));
+            combine_columns<KMAX, CPL>(v, gs, rows, p.k, res != nullptr, r, out);
+            uint32_t packed[CPL / 2];
+#pragma unroll
+            for (int c = 0; c < CPL / 2; ++c) packed[c] = pack_bf16x2(out[2 * c], out[2 * c + 1]);
+            __nv_bfloat16* dst = y + (int64_t)t * p.n_out + col;
+            if constexpr (CPL >= 8) {
+#pragma unroll
+                for (int c = 0; c < CPL / 8; ++c)
+                    reinterpret_cast<uint4*>(dst)[c] = make_uint4(
+                        packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+            } else {
+                *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+            }
         }
     }
 }
@@ -712,11 +752,12 @@ constexpr int kPairStageBytes = kABytes + kPairBBoxes * kBBoxBytes;   // 32 KB
 constexpr size_t kPairSmemBytes = (size_t)kPairStages * kPairStageBytes + kEpiBytes + 1024;
 constexpr int kPairMinRows = 512;
 // Rounds of GEMM2 pair tiles from which the combine runs in GEMM2's epilogue.
-// Finishing y there made GEMM2 longer by about as much as the combine kernel
-// took at the Mixtral prefill batch (7 rounds: +27-31 us against 34-36 us, a
-// variant that only counted cost +2 us), and saved 40-95 us a step at the
-// skewed 16384-token batch (28 rounds).
-constexpr int kFuseMinRounds = 16;
+// The finishing of a pair's last tile is not hidden behind a next tile: with
+// one round (the quarter-width batch) GEMM2 grew by 22 us against an 8 us
+// combine; at the Mixtral prefill batch (7 rounds) the step measured 8-18 us
+// shorter than with the separate combine, at the skewed 16384-token batch
+// (28 rounds) 40-95 us.
+constexpr int kFuseMinRounds = 4;
 constexpr int kPairMinRounds = 8;
 constexpr int kInlineHalfRounds = 16;
 
@@ -1036,9 +1077,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int ncols = pt.half ? boxes * kBoxN : 2 * boxes * kBoxN;
                 const int x0 = pt.ti.n0 + col_half * boxes * kBoxN;
                 if (p.k <= 2)
-                    finish_tokens<2>(p, st.base, valid, tma, grow, x0, ncols, lane);
+                    finish_tokens<2, 8>(p, st.base, valid, tma, grow, x0, ncols, lane);
                 else
-                    finish_tokens<8>(p, st.base, valid, tma, grow, x0, ncols, lane);
+                    finish_tokens<8, 32>(p, st.base, valid, tma, grow, x0, ncols, lane);
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
@@ -1213,7 +1254,7 @@ bool combine_fusable(const moe_shape& s) {
     return (int64_t)s.T * s.k >= gemm::kPairMinRows && s.d % 256 == 0;
 }
 
-// The combine is fused only when GEMM2 has many rounds of pair tiles
+// The combine is fused only when GEMM2 has several rounds of pair tiles
 // (kFuseMinRounds).
 bool combine_fused(const moe_shape& s) {
     if (!combine_fusable(s)) return false;

@@ -70,10 +70,11 @@ def test_workspace_sizes():
 
 
 def test_forward_kernel_count():
-    """Six kernels, five once the down projection forms y itself (16 or more
+    """Six kernels, five once the down projection forms y itself (4 or more
     rounds of its CTA-pair tiles; the host without a GPU assumes the B200's
     148 SMs, 74 pairs), none for an empty batch, an error for a rejected shape."""
-    assert moe.moe_forward_kernel_count((4096, 4096, 14336, 8, 2)) == 6    # 512 pair tiles
+    assert moe.moe_forward_kernel_count((4096, 4096, 14336, 8, 2)) == 5    # 512 pair tiles
+    assert moe.moe_forward_kernel_count((1024, 1024, 3584, 8, 2)) == 6     # 32 pair tiles
     assert moe.moe_forward_kernel_count((16, 4096, 14336, 8, 2)) == 6      # single CTAs
     assert moe.moe_forward_kernel_count((16384, 4096, 14336, 8, 2)) == 5   # 2048 pair tiles
     assert moe.moe_forward_kernel_count((50600, 384, 256, 8, 2)) == 6      # d not a multiple of 256

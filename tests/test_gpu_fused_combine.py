@@ -1,14 +1,15 @@
 """The combine fused into the down projection's epilogue, bit for bit.
 
 When a routed batch gives the down projection (on CTA pairs, 256-row and
-256-column tiles, d a multiple of 256) at least 16 rounds of pair tiles on the
+256-column tiles, d a multiple of 256) at least 4 rounds of pair tiles on the
 device's SMs, that GEMM forms y itself: the last of a token's k row tiles to
 store its o rows adds the token's gate-weighted rows up.  That y must have
 exactly the bits of the separate path (dispatch, experts, combine through
 their own entry points), and of a float32 model of the combine's arithmetic
 written here in numpy: products rounded to float32, summed in slot order, the
 block's residual added last, one rounding to bf16 (nearest even).  The cases
-below have 1184 or more pair tiles (16 rounds of 74 pairs on 148 SMs) unless
+below have 1184 or more pair tiles (16 rounds of 74 pairs on 148 SMs, well past
+the 4 from which the down projection forms y) unless
 marked otherwise.
 """
 import numpy as np
@@ -32,10 +33,10 @@ CASES = {
     "E16k4": (4800, 4096, 256, 16, 4, 36, False),
     "E32k8": (4800, 2048, 256, 32, 8, 37, False),      # the largest E and k (and d for E = 32)
     "E1k1": (19044, 4096, 256, 1, 1, 38, False),       # 74 full pair tiles and a half tile
-    # not fused: d not a multiple of 256, fewer than 512 rows, under 16 rounds
+    # not fused: d not a multiple of 256, fewer than 512 rows, under 4 rounds
     "d384": (1400, 384, 256, 8, 2, 39, False),
     "small": (200, 256, 256, 8, 2, 40, False),
-    "rounds": (4096, 4096, 256, 8, 2, 41, False),      # the prefill batch's 7 rounds
+    "rounds": (1024, 1024, 256, 8, 2, 41, False),      # the quarter-width batch: 32 tiles
 }
 
 
