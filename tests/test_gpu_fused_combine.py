@@ -204,16 +204,16 @@ def test_fused_combine_with_expert_biases():
 
 
 def test_fused_combine_in_token_chunks_equals_the_whole_batch():
-    """moe_forward_hostio cuts a batch of 20000 tokens into chunks of 2496, 15008
-    and 2496 tokens: the middle chunk forms y inside GEMM2, the edge chunks (304
-    pair tiles each) run the combine kernel, and the whole batch (2496 tiles) is
-    fused too; y must be the same bits either way."""
-    T, d, d_ff, E, k = 20000, 4096, 256, 8, 2
+    """moe_forward_hostio cuts a batch of 18000 tokens into chunks of 2240, 13520
+    and 2240 tokens: the middle chunk (1680 pair tiles) forms y inside GEMM2, the
+    edge chunks (272 pair tiles each, under 4 rounds) run the combine kernel, and
+    the whole batch (2240 tiles) is fused too; y must be the same bits either way."""
+    T, d, d_ff, E, k = 18000, 4096, 256, 8, 2
     inp = make_inputs(T, d, d_ff, E, k, 42, bias=True)
     shape = inp["shape"]
     assert moe.moe_forward_kernel_count(shape) == 5
-    assert moe.moe_forward_kernel_count((15008, d, d_ff, E, k)) == 5
-    assert moe.moe_forward_kernel_count((2496, d, d_ff, E, k)) == 6
+    assert moe.moe_forward_kernel_count((13520, d, d_ff, E, k)) == 5
+    assert moe.moe_forward_kernel_count((2240, d, d_ff, E, k)) == 6
     dev = to_dev(inp)
     y = moe.moe_forward(shape, dev["x"], dev["Wg"], dev["bias"], dev["W1"], dev["W3"], dev["W2"])
     x_host = inp["x"].clone().pin_memory()
